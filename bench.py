@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Throughput of the top-k MoE FFN forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+One step = one whole forward (router, permutation, both grouped GEMMs,
+combine) over one batch of synthetic tokens, through the C ABI.  The default
+workload is the Mixtral-8x7B-shaped bf16 layer (T=4096 tokens, D=4096,
+F=14336, E=8, top_k=2), the configuration the bf16-peak target is quoted on.
+With N > 1 (torchrun) each rank runs an independent replica on its own GPU
+(tokens are independent: no collective on the data path); the timing is the
+max over ranks and ``value`` counts every rank's tokens.
+
+Printed: one JSON line (rank 0) with tokens/s (``value``), routed TFLOP/s,
+``roofline`` of the dominant kernel (timed live with CUDA events on the
+launching stream), ``e2e`` (pinned host buffers, copies inside the timed
+region), ``cpu_baseline`` (the float64 oracle on a bounded token sample on
+this host's cores), ``clocks`` sampled through NVML during the timed region.
+
+``--impl reference`` times the float64 oracle (the only reference this
+subject has) on the same workload, on host cores, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-FFN fwd tokens/s + routed TFLOP/s (% B200 bf16 peak; % HBM at small T)"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "source": "fallback"}
+NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+L2_BYTES = 126 * 1024 * 1024
+KERNELS_PER_FORWARD = 6   # router, permute scan, permute scatter, gate_up, down, combine
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS)
+
+
+def source_hash() -> str:
+    """Hash of the grouped-GEMM source: a stored DRAM-traffic figure is only
+    reported while it matches the kernel it was taken on."""
+    h = hashlib.sha256()
+    for f in ("gemm_tc.cu", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "mixture_experts_ffn_09_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(workload: str, kernel: str):
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(p))
+        e = d[workload][kernel]
+        if e.get("source_hash") == source_hash():
+            return float(e["bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML (read only)."""
+
+    NAMES = {"nvmlClocksEventReasonGpuIdle": "gpu_idle",
+             "nvmlClocksEventReasonApplicationsClocksSetting": "applications_clocks_setting",
+             "nvmlClocksEventReasonSwPowerCap": "sw_power_cap",
+             "nvmlClocksEventReasonHwSlowdown": "hw_slowdown",
+             "nvmlClocksEventReasonSyncBoost": "sync_boost",
+             "nvmlClocksEventReasonSwThermalSlowdown": "sw_thermal_slowdown",
+             "nvmlClocksEventReasonHwThermalSlowdown": "hw_thermal_slowdown",
+             "nvmlClocksEventReasonHwPowerBrakeSlowdown": "hw_power_brake_slowdown",
+             "nvmlClocksEventReasonDisplayClockSetting": "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml as N
+            self.N = N
+            N.nvmlInit()
+            self.h = N.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self.t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        N = self.N
+        while not self._stop.is_set():
+            try:
+                self.samples.append(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
+                bits = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for attr, name in self.NAMES.items():
+                    v = getattr(N, attr, None)
+                    if v is not None and bits & v:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t.start()
+
+    def stop(self) -> dict:
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        self._stop.set()
+        self.t.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------- accounting
+def routed_flops(w, K=None) -> float:
+    return w.routed_flops() if K is None else w.with_K(K).routed_flops()
+
+
+def gate_up_flops(w) -> float:
+    return float((4 if w.act == "silu_gated" else 2) * w.R * w.D * w.F)
+
+
+def algorithmic_bytes(w, touched: int) -> float:
+    """Weights of the experts actually selected, x in, out, selections and
+    weights; the expert-sorted copies and intermediates are overhead."""
+    s = 2 if w.dtype == "bf16" else 4
+    gu_rows = 2 * w.F if w.act == "silu_gated" else w.F
+    weights = touched * (gu_rows * w.D + w.D * w.F) * s + w.E * w.D * s
+    return float(weights + 2 * w.T * w.D * s + w.T * w.K * 12)
+
+
+def gate_up_bytes(w, touched: int) -> float:
+    s = 2 if w.dtype == "bf16" else 4
+    gu_rows = 2 * w.F if w.act == "silu_gated" else w.F
+    return float(touched * gu_rows * w.D * s + w.R * w.D * s + w.R * w.F * s)
+
+
+# ------------------------------------------------------------ oracle timing
+def oracle_rate(w, d, budget_s: float, first_n: int = 8):
+    """Tokens/s of the float64 oracle (dense over all experts, as it stands)
+    on a bounded token sample.  Returns (tokens_per_s, n_tokens, seconds)."""
+    import numpy as np
+    from oracle import moe_oracle as O
+    from mixture_experts_ffn_09_b200 import synth
+    x = synth.as_float32(d["x"]).reshape(-1, w.D)
+    gu = synth.as_float32(d["gate_up_proj"]).astype(np.float64)
+    dn = synth.as_float32(d["down_proj"]).astype(np.float64)
+    rt = synth.as_float32(d["router"]).astype(np.float64)
+
+    def run(n):
+        t0 = time.perf_counter()
+        O.moe_ffn_forward(x[:n], rt, gu, dn, w.K, w.norm_topk_prob, w.act, d["router_bias"],
+                          d["b1"], d["b2"])
+        return time.perf_counter() - t0
+
+    n = min(first_n, w.T)
+    t = run(n)
+    if t < budget_s / 3 and n < w.T:
+        n = int(min(w.T, max(n + 1, n * (budget_s / max(t, 1e-6)))))
+        t = run(n)
+    return n / t, n, t
+
+
+def cpu_cores() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        nt = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if nt:
+            return int(max(nt))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------- ranks
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank number over all ranks (identity at world 1)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def init_dist(world: int, backend: str):
+    if world <= 1:
+        return
+    import datetime
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def workload_config(w, world: int) -> dict:
+    return {"workload": w.name, "T": w.T, "D": w.D, "F": w.F, "E": w.E, "K": w.K, "act": w.act,
+            "norm_topk_prob": w.norm_topk_prob, "tokens_per_gpu": w.T,
+            "global_batch_tokens": w.T * world,
+            "parallelism": "replicas" if world > 1 else "single-gpu",
+            "l2": "inputs larger than L2 (expert weights streamed every step)"
+            if algorithmic_bytes(w, w.E) > L2_BYTES else "L2 not flushed (inputs fit in L2)"}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, w):
+    import numpy as np
+    import torch
+    from mixture_experts_ffn_09_b200 import build, moe, synth
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    init_dist(world, "nccl")
+    build.build()
+    dev = torch.device("cuda", local)
+    d = synth.make_inputs(w)
+
+    def up(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    x, router, gu, dn = up(d["x"]), up(d["router"]), up(d["gate_up_proj"]), up(d["down_proj"])
+    rb, b1, b2 = up(d["router_bias"]), up(d["b1"]), up(d["b2"])
+    x = x.reshape(w.T, w.D)
+    dt = moe.BF16 if w.dtype == "bf16" else moe.F32
+    act = moe.ACT_NAMES[w.act]
+    ws = torch.empty(moe.workspace_size(w.T, w.D, w.F, w.E, w.K, dt, act), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty_like(x)
+    sel = torch.empty(w.T, w.K, dtype=torch.int64, device=dev)
+    wts = torch.empty(w.T, w.K, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(xin=x, o=out):
+        moe.ffn_forward(xin, router, gu, dn, w.E, w.K, w.norm_topk_prob, act, o, sel, wts, rb, b1,
+                        b2, None, ws, stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    st = moe.device_status(stream)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status after warm-up: {moe.status_string(st)}")
+    load = np.bincount(sel.cpu().numpy().ravel(), minlength=w.E)
+    touched = int((load > 0).sum())
+
+    # ---------------- timed region: K forwards, device events on the stream
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    moe.profile_enable(True)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    stage_ms, calls = moe.profile_read()
+    moe.profile_enable(False)
+    local_ms = t0.elapsed_time(t1)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    ms = max_over_ranks(local_ms, world, dev)
+    ms_step = ms / args.steps
+    tokens_per_s = world * w.T / (ms_step / 1e3)
+    st = moe.device_status(stream)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status after timing: {moe.status_string(st)}")
+
+    # ---------------- end to end: pinned host x in, out back, every step
+    xh = torch.from_numpy(np.ascontiguousarray(d["x"]).view(np.int16 if dt == moe.BF16 else np.float32))
+    xh = (xh.view(torch.bfloat16) if dt == moe.BF16 else xh).reshape(w.T, w.D).pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    xd = torch.empty_like(x)
+    e_steps = max(1, min(args.steps, 200))
+    for _ in range(2):
+        xd.copy_(xh, non_blocking=True)
+        step(xd, out)
+        oh.copy_(out, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        xd.copy_(xh, non_blocking=True)
+        step(xd, out)
+        oh.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e_steps
+    io_bytes = w.T * w.D * (2 if dt == moe.BF16 else 4)
+
+    # ---------------- roofline of the dominant kernel (gate_up)
+    peaks = load_peaks()
+    per_call = {k: v / max(calls, 1) for k, v in stage_ms.items()}
+    dom = max(per_call, key=per_call.get)
+    t_gu = per_call["gate_up"] / 1e3
+    hbm_bound = w.T * w.K <= 512
+    if hbm_bound:
+        achieved = gate_up_bytes(w, touched) / t_gu / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"kernel": "grouped_gemm_tc<silu_gated> (gate_up)", "bound": "hbm",
+                "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": peaks["source"] + " hbm copy",
+                "algorithmic_bytes_per_launch": gate_up_bytes(w, touched)}
+    else:
+        achieved = gate_up_flops(w) / t_gu / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"kernel": "grouped_gemm_tc<silu_gated> (gate_up)", "bound": "tensor",
+                "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4),
+                "peak_source": peaks["source"] + " bf16 sustained (kernel timed inside a long loop)",
+                "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4),
+                "frac_of_datasheet_2250": round(achieved / NOMINAL["bf16_tflops"], 4),
+                "algorithmic_flops_per_launch": gate_up_flops(w)}
+    roof["traffic"] = stored_traffic(w.name, "gate_up")
+    roof["avg_launch_ms"] = round(per_call["gate_up"], 4)
+
+    rflops = routed_flops(w)
+    abytes = algorithmic_bytes(w, touched)
+    result = {
+        "metric": METRIC, "value": round(tokens_per_s, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded, shapes of the pages' workloads; random-init weights)",
+        "config": workload_config(w, world),
+        "routed_tflops": round(world * rflops / (ms_step / 1e3) / 1e12, 2),
+        "frac_of_bf16_peak": {
+            "measured_burst": round(rflops / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+            "measured_sustained": round(rflops / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops_sustained"], 4),
+            "datasheet_2250": round(rflops / (ms_step / 1e3) / 1e12 / NOMINAL["bf16_tflops"], 4)},
+        "hbm": {"algorithmic_gb_per_step": round(abytes / 1e9, 4),
+                "achieved_gbs": round(abytes / (ms_step / 1e3) / 1e9, 1),
+                "frac_of_measured": round(abytes / (ms_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                "frac_of_nominal_8tbs": round(abytes / (ms_step / 1e3) / 1e9 / NOMINAL["hbm_gbs"], 4)},
+        "stages_ms": {k: round(v, 4) for k, v in per_call.items()},
+        "dominant_stage": dom,
+        "expert_load": load.tolist(), "experts_touched": touched,
+        "roofline": roof,
+        "e2e": {"value": round(world * w.T / (e_ms / 1e3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
+                "ms_per_step": round(e_ms, 4),
+                "how": "pinned host x -> device, moe_ffn_forward, out -> pinned host, one stream"},
+        "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, n, secs = oracle_rate(w, d, args.cpu_seconds)
+        result["cpu_baseline"] = {"value": round(rate, 4), "unit": UNIT, "cores": cpu_cores(),
+                                  "kind": "oracle",
+                                  "sample": f"first {n} tokens of the workload, dense over all "
+                                            f"{w.E} experts in float64 ({secs:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------- reference arm
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    from mixture_experts_ffn_09_b200 import synth
+    d = synth.make_inputs(w)
+    # one step = the oracle on a bounded token sample; size it so that the
+    # whole run stays within a few minutes
+    total = args.steps + args.warmup
+    rate0, n0, t0 = oracle_rate(w, d, budget_s=1.0, first_n=2)
+    per_step_s = max(0.5, min(20.0, 150.0 / max(total, 1)))
+    n = int(max(1, min(w.T, rate0 * per_step_s)))
+    import numpy as np
+    from oracle import moe_oracle as O
+    x = synth.as_float32(d["x"]).reshape(-1, w.D)
+    gu = synth.as_float32(d["gate_up_proj"]).astype(np.float64)
+    dn = synth.as_float32(d["down_proj"]).astype(np.float64)
+    rt = synth.as_float32(d["router"]).astype(np.float64)
+
+    def step(i):
+        lo = (i * n) % max(w.T - n + 1, 1)
+        O.moe_ffn_forward(x[lo:lo + n], rt, gu, dn, w.K, w.norm_topk_prob, w.act, d["router_bias"],
+                          d["b1"], d["b2"])
+
+    for i in range(args.warmup):
+        step(i)
+    t = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    secs = time.perf_counter() - t
+    rate = args.steps * n / secs
+    cores = cpu_cores()
+    sample = (f"{n} tokens per step (of {w.T}), dense over all {w.E} experts in float64, "
+              f"{args.steps} steps in {secs:.1f} s")
+    print(json.dumps({
+        "metric": METRIC, "value": round(rate, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / max(args.steps, 1) * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, shapes of the pages' workloads; random-init weights)",
+        "config": workload_config(w, 1), "impl": "reference",
+        "cpu_baseline": {"value": round(rate, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(rate, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    from mixture_experts_ffn_09_b200 import synth
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=synth.MIXTRAL.name, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle sample (cpu_baseline)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

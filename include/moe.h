@@ -1,0 +1,182 @@
+/*
+ * libmoe — forward pass of a top-k mixture-of-experts feed-forward layer on
+ * one NVIDIA B200 (sm_100a).  Plain C ABI: device pointers, sizes, a stream
+ * handle passed as void* (a cudaStream_t, NULL = the legacy default stream).
+ *
+ * What is computed (for each token t of x, flattened to (T, D)):
+ *
+ *   logits[t, e] = sum_d x[t, d] * router[e, d] (+ router_bias[e])
+ *   p[t, :]      = softmax(logits[t, :]) over the E experts
+ *   idx[t, 0..K) = the K largest p, in descending order, equal scores going
+ *                  to the lower expert index
+ *   w[t, k]      = p[t, idx[t, k]] / (sum_j p[t, idx[t, j]] + 1e-9)
+ *                  when norm_topk_prob, else p[t, idx[t, k]]
+ *   out[t, :]    = sum_k w[t, k] * expert_{idx[t, k]}(x[t, :])
+ *
+ * with expert_e either
+ *   MOE_ACT_SILU_GATED:  down_e(silu(gate_e x) * up_e x)   (no biases), or
+ *   MOE_ACT_RELU:        W2_e relu(W1_e x + b1_e) + b2_e.
+ *
+ * Sources, by page and section:
+ *   - "Mixture-of-Experts FFN" (crackedaicode.com Flax exercise): "Compute
+ *     the experts and router" (Dense/ReLU experts, biased Dense(E) router,
+ *     softmax, top_k order and ties), "Weight the selected outputs" (the
+ *     1e-9 renormalisation and the per-token gather), "Problem" (shapes,
+ *     1 <= K <= E, positive dimensions, features fastest).
+ *   - "mojolearn.MoEBlock": class description (SiLU-gated Mixtral expert,
+ *     lower-index ties, forward only), "Variables" (router (E, D),
+ *     gate_up_proj (E, 2F, D), down_proj (E, D, F), selected_experts int64),
+ *     "Parameters" (top_k range -> error, hidden_act other than silu ->
+ *     error, norm_topk_prob), forward(x) (float64 input -> error, output
+ *     with the shape of x).
+ *   - "Mixture of experts" (dewml.dev), "Expert computation and placement":
+ *     tokens are sorted into expert order and the experts run as one grouped
+ *     matrix multiplication; each contraction accumulates in at least fp32
+ *     and rounds once to the compute dtype.
+ *
+ * Only the selected experts are computed.  Work runs asynchronously on the
+ * given stream; results are deterministic (bitwise repeatable run to run:
+ * no floating-point atomics anywhere).  The library allocates nothing and
+ * keeps no state between calls except the optional stage profiler and a
+ * per-device error word written by bounded waits (see moe_device_status).
+ */
+#ifndef LIBMOE_MOE_H
+#define LIBMOE_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,      /* K outside [1, E], a dimension <= 0, a required pointer NULL
+                                   ("Problem": positive dimensions, 1 <= K <= E;
+                                   mojolearn "Parameters": top_k range -> ValueError) */
+  MOE_ERR_UNSUPPORTED_ACT = 2,  /* act is neither SiLU-gated nor ReLU (mojolearn "Parameters":
+                                   hidden_act other than silu -> NotImplementedError) */
+  MOE_ERR_DTYPE = 3,            /* dtype other than f32 / bf16, e.g. MOE_F64 (mojolearn
+                                   forward(x): float64 input -> TypeError) */
+  MOE_ERR_SHAPE = 4,            /* a size the kernels cannot index (E > MOE_MAX_EXPERTS,
+                                   T*K or T*max(D,F) beyond 2^31-1) */
+  MOE_ERR_ALIGNMENT = 5,        /* a device pointer not 16-byte aligned, or on the bf16 path D or F
+                                   not a multiple of 8 (tensor-memory-access rows need 16-byte
+                                   strides) */
+  MOE_ERR_WORKSPACE = 6,        /* workspace NULL or smaller than moe_ffn_workspace_size() */
+  MOE_ERR_CUDA = 7,             /* a CUDA runtime call failed (a launch error, or a sticky error
+                                   from earlier work on the device); see moe_last_error() */
+  MOE_ERR_TIMEOUT = 8,          /* a bounded wait inside a kernel gave up (reported by
+                                   moe_device_status); outputs of that call are undefined */
+  MOE_ERR_DEVICE = 9            /* the current device is not sm_100 (B200 / GB200) */
+} moe_status_t;
+
+typedef enum {
+  MOE_ACT_SILU_GATED = 0,  /* Mixtral expert: gate_up_proj (E, 2F, D), rows [0,F) gate, [F,2F) up;
+                              down_proj (E, D, F); b1, b2 must be NULL */
+  MOE_ACT_RELU = 1         /* exercise expert: gate_up_proj slot holds W1 (E, F, D), down_proj slot
+                              holds W2 (E, D, F); b1 (E, F) and b2 (E, D) required */
+} moe_act_t;
+
+typedef enum {
+  MOE_F32 = 0,   /* float32 x / weights / out; experts in fp32 FMA on CUDA cores */
+  MOE_BF16 = 1,  /* bfloat16 x / weights / out; tensor cores, fp32 accumulation, the
+                    intermediate H = act(...) rounded once to bf16 */
+  MOE_F64 = 2    /* not supported: always MOE_ERR_DTYPE */
+} moe_dtype_t;
+
+/* Largest expert count the router kernel holds in registers. */
+#define MOE_MAX_EXPERTS 256
+
+/*
+ * Bytes of device workspace moe_ffn_forward needs for these sizes (0 when
+ * the sizes are invalid).  Holds the token permutation, the expert-sorted
+ * copy of x, the intermediate H (T*K, F) and per-slot expert outputs
+ * (T*K, D).  The caller allocates it; contents need not be initialised and
+ * are garbage after the call.  Calls that share a workspace must not
+ * overlap on the GPU.
+ */
+MOE_API size_t moe_ffn_workspace_size(int64_t T, int64_t D, int64_t F, int E, int K,
+                              moe_dtype_t dt, moe_act_t act);
+
+/*
+ * The whole forward.  All pointers are device pointers owned by the caller,
+ * 16-byte aligned, row-major with the last dimension contiguous:
+ *
+ *   x                (T, D)            dt    tokens; any leading shape flattened to T
+ *   router           (E, D)            dt    router weight, one row per expert
+ *   gate_up_proj     (E, 2F, D) / (E, F, D)  dt   see moe_act_t
+ *   down_proj        (E, D, F)         dt
+ *   out              (T, D)            dt    written once per element (must not alias inputs)
+ *   selected_experts (T, K)            int64 may be NULL
+ *   routing_weights  (T, K)            f32   may be NULL
+ *   router_bias      (E)               f32   may be NULL for SiLU; required for ReLU
+ *   b1               (E, F)            f32   ReLU only
+ *   b2               (E, D)            f32   ReLU only
+ *   router_logits    (T, E)            f32   may be NULL
+ *   workspace        workspace_bytes         >= moe_ffn_workspace_size(...)
+ *
+ * Host-side validation happens before any launch; on an error nothing is
+ * launched and no output is touched.  Returns MOE_OK once all kernels are
+ * enqueued on `stream`; inputs must stay valid until the stream reaches
+ * that point.
+ */
+MOE_API moe_status_t moe_ffn_forward(const void* x, const void* router, const void* gate_up_proj,
+                             const void* down_proj, int E, int K, int norm_topk_prob,
+                             moe_act_t act, void* out, int64_t* selected_experts,
+                             float* routing_weights, int64_t T, int64_t D, int64_t F,
+                             moe_dtype_t dt, const float* router_bias, const float* b1,
+                             const float* b2, float* router_logits, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
+ * Router only: logits, softmax, top-k selection and weights (the first half
+ * of moe_ffn_forward, same definitions).  router_logits may be NULL;
+ * selected_experts and routing_weights are required.  Needs no workspace.
+ */
+MOE_API moe_status_t moe_route(const void* x, const void* router, const float* router_bias, int64_t T,
+                       int64_t D, int E, int K, int norm_topk_prob, moe_dtype_t dt,
+                       float* router_logits, int64_t* selected_experts, float* routing_weights,
+                       void* stream);
+
+/* Short English description of a status code (static storage). */
+MOE_API const char* moe_status_string(moe_status_t status);
+
+/* Detail of the last error returned on this host thread ("" if none). */
+MOE_API const char* moe_last_error(void);
+
+/* MOE_ABI_VERSION of the built library. */
+MOE_API int moe_abi_version(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error
+ * word, which kernels set when a bounded wait gives up instead of hanging.
+ * Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_CUDA.
+ */
+MOE_API moe_status_t moe_device_status(void* stream);
+
+/*
+ * Stage profiler.  While enabled, moe_ffn_forward records CUDA events
+ * around each of its kernels on the caller's stream (router, permute,
+ * gate_up, down, combine).  moe_profile_read synchronises on the recorded
+ * events, adds their durations (milliseconds) into ms[0..n_stages) and
+ * returns the number of forward calls covered, then resets the counters.
+ */
+#define MOE_NUM_STAGES 5
+MOE_API moe_status_t moe_profile_enable(int enable);
+MOE_API int moe_profile_read(float* ms, int n_stages);
+MOE_API const char* moe_stage_name(int stage);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LIBMOE_MOE_H */

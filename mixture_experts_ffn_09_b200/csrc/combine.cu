@@ -1,0 +1,95 @@
+// Weighted combine: out[t, :] = sum_k w[t, k] * Y[pos[t, k], :].
+//
+// "Mixture-of-Experts FFN" (crackedaicode.com Flax exercise), section
+// "Weight the selected outputs": each token sums its own K selected expert
+// outputs weighted by its routing weights.  Y holds one row per (token,
+// slot) in expert order; pos maps a slot to its row.  Each output element
+// is written exactly once, the K terms are summed in fp32 in slot order and
+// rounded once to the output dtype: no atomics, bitwise repeatable.
+//
+// HBM-bound gather: one CTA per token, 16-byte loads and stores.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 128;
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) combine_bf16_kernel(const __nv_bfloat16* __restrict__ Y,
+                                                                const float* __restrict__ w,
+                                                                const int* __restrict__ pos, int K,
+                                                                int D,
+                                                                __nv_bfloat16* __restrict__ out) {
+  __shared__ int sp[kMaxExperts];
+  __shared__ float sw[kMaxExperts];
+  const int t = blockIdx.x;
+  for (int k = threadIdx.x; k < K; k += kThreads) {
+    sp[k] = pos[static_cast<size_t>(t) * K + k];
+    sw[k] = w[static_cast<size_t>(t) * K + k];
+  }
+  __syncthreads();
+  for (int d = threadIdx.x * 8; d < D; d += kThreads * 8) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int k = 0; k < K; ++k) {
+      float y[8];
+      load8(Y + static_cast<size_t>(sp[k]) * D + d, y);
+      const float wk = sw[k];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(wk, y[i], acc[i]);
+    }
+    uint4 o;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    *reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * D + d) = o;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) combine_f32_kernel(const float* __restrict__ Y,
+                                                               const float* __restrict__ w,
+                                                               const int* __restrict__ pos, int K,
+                                                               int D, float* __restrict__ out) {
+  __shared__ int sp[kMaxExperts];
+  __shared__ float sw[kMaxExperts];
+  const int t = blockIdx.x;
+  for (int k = threadIdx.x; k < K; k += kThreads) {
+    sp[k] = pos[static_cast<size_t>(t) * K + k];
+    sw[k] = w[static_cast<size_t>(t) * K + k];
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < D; d += kThreads) {
+    float acc = 0.f;
+    for (int k = 0; k < K; ++k) acc = fmaf(sw[k], __ldg(Y + static_cast<size_t>(sp[k]) * D + d), acc);
+    out[static_cast<size_t>(t) * D + d] = acc;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const void* Y, const float* w32, const int* pos, int T, int K, int D,
+                           int dt, void* out, cudaStream_t s) {
+  if (dt == kBF16) {
+    combine_bf16_kernel<<<T, kThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(Y), w32, pos, K,
+                                               D, static_cast<__nv_bfloat16*>(out));
+  } else {
+    combine_f32_kernel<<<T, kThreads, 0, s>>>(static_cast<const float*>(Y), w32, pos, K, D,
+                                              static_cast<float*>(out));
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,62 @@
+// Internal launch interface between the C ABI (moe_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kMaxExperts = 256;
+constexpr int kRouterTokensPerCta = 32;   // tokens per router CTA = per permute block
+constexpr int kTileM = 128;               // rows of one grouped-GEMM tile
+
+enum DType : int { kF32 = 0, kBF16 = 1 };
+
+struct RouteArgs {
+  const void* x;            // (T, D) f32 or bf16
+  const void* router;       // (E, D)
+  const float* router_bias; // (E) or null
+  int T, D, E, K, norm, dt;
+  float* logits;            // (T, E) or null
+  int64_t* sel64;           // (T, K) or null
+  float* wout;              // (T, K) or null
+  int* idx32;               // (T, K) or null
+  float* w32;               // (T, K) or null
+  int* blockcounts;         // (ceil(T / kRouterTokensPerCta), E) or null
+};
+
+cudaError_t launch_router(const RouteArgs& a, cudaStream_t s);
+
+// Per-expert totals -> offsets (E + 1) and each router block's first row
+// per expert, blockbase (B, E).
+cudaError_t launch_permute_scan(const int* blockcounts, int B, int E, int* offsets,
+                                int* blockbase, cudaStream_t s);
+
+// Stable scatter of the (token, slot) pairs into expert order: perm[row] =
+// slot, pos[slot] = row, and x_perm[row, :] = x[slot / K, :].
+cudaError_t launch_permute_scatter(const int* idx32, const int* blockbase, int T, int K, int E,
+                                   const void* x, int D, int elem_bytes, int* perm, int* pos,
+                                   void* x_perm, cudaStream_t s);
+
+// out[t, :] = sum_k w[t, k] * Y[pos[t, k], :], fp32 sum in k order.
+cudaError_t launch_combine(const void* Y, const float* w32, const int* pos, int T, int K, int D,
+                           int dt, void* out, cudaStream_t s);
+
+// fp32 grouped GEMMs on CUDA cores (the float32 path).
+//   act 0: H = silu(A W_gate^T) * (A W_up^T)   (W rows [0,N) gate, [N,2N) up)
+//   act 1: H = relu(A W^T + bias)
+//   act 2: H = A W^T (+ bias)
+cudaError_t launch_gemm_simt_f32(int act, const float* A, const float* W, const int* offsets,
+                                 int E, int T, int Kdim, int N, int w_rows_per_expert,
+                                 const float* bias, float* C, cudaStream_t s);
+
+// bf16 grouped GEMMs on the tcgen05 tensor cores (same three epilogues).
+// A: (a_rows, Kdim) bf16 sorted rows; W: (E * w_rows_per_expert, Kdim) bf16.
+cudaError_t launch_gemm_tc(int act, const void* A, int a_rows, const void* W, const int* offsets,
+                           int E, int T, int Kdim, int N, int w_rows_per_expert,
+                           const float* bias, void* C, unsigned int* err, cudaStream_t s);
+
+int num_sms();
+
+}  // namespace moe

@@ -1,0 +1,421 @@
+// libmoe C ABI: argument validation, workspace layout, the launch sequence
+// of one forward, device status and the optional stage profiler.
+//
+// One forward = five stages on the caller's stream:
+//   router   logits, softmax, top-k, weights, per-block expert histogram
+//   permute  expert offsets (1-CTA scan) + stable scatter and row gather
+//   gate_up  grouped GEMM 1 with the activation fused in its epilogue
+//   down     grouped GEMM 2 (+ b2 for the Dense/ReLU expert)
+//   combine  weighted gather back to token order, one write per element
+#include <limits.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+__device__ unsigned int g_device_error;   // per device: bounded waits that gave up
+
+moe_status_t fail(moe_status_t s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+moe_status_t fail(moe_status_t s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+moe_status_t cuda_fail(cudaError_t e, const char* where) {
+  return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ------------------------------------------------------------ device info
+struct DevInfo {
+  bool init = false;
+  int sms = 0;
+  int major = 0, minor = 0;
+  unsigned int* err = nullptr;
+};
+std::mutex g_dev_mu;
+DevInfo g_dev[64];
+
+moe_status_t device_info(DevInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(MOE_ERR_DEVICE, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.init) {
+    if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev)) !=
+            cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev)) !=
+            cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_device_error)) != cudaSuccess)
+      return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+    d.err = static_cast<unsigned int*>(p);
+    d.init = true;
+  }
+  if (d.major != 10 || d.minor != 0)
+    return fail(MOE_ERR_DEVICE, "device %d is sm_%d%d; libmoe is built for sm_100a", dev, d.major,
+                d.minor);
+  *out = &d;
+  return MOE_OK;
+}
+
+// --------------------------------------------------------------- profiler
+struct ProfState {
+  bool enabled = false;
+  int calls = 0;
+  std::vector<cudaEvent_t> pool;
+  std::vector<std::pair<int, std::pair<cudaEvent_t, cudaEvent_t>>> recs;   // stage, (start, end)
+  size_t next = 0;
+};
+std::mutex g_prof_mu;
+ProfState g_prof;
+
+cudaEvent_t prof_event() {
+  if (g_prof.next == g_prof.pool.size()) {
+    cudaEvent_t ev;
+    if (cudaEventCreate(&ev) != cudaSuccess) return nullptr;
+    g_prof.pool.push_back(ev);
+  }
+  return g_prof.pool[g_prof.next++];
+}
+
+struct StageTimer {
+  bool on;
+  cudaStream_t s;
+  explicit StageTimer(cudaStream_t st) : on(false), s(st) {
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    on = g_prof.enabled;
+    if (on) g_prof.calls++;
+  }
+  // Records an event pair around fn() on the stream when profiling.
+  template <typename Fn>
+  cudaError_t run(int stage, Fn fn) {
+    if (!on) return fn();
+    cudaEvent_t a, b;
+    {
+      std::lock_guard<std::mutex> lock(g_prof_mu);
+      a = prof_event();
+      b = prof_event();
+      if (a && b) g_prof.recs.push_back({stage, {a, b}});
+    }
+    if (a) cudaEventRecord(a, s);
+    cudaError_t e = fn();
+    if (b) cudaEventRecord(b, s);
+    return e;
+  }
+};
+
+// ------------------------------------------------------ workspace layout
+struct Layout {
+  size_t idx32, w32, bcount, bbase, offsets, perm, pos, xperm, h, y, total;
+  int B, Rpad;
+};
+
+Layout layout(int64_t T, int64_t D, int64_t F, int E, int K, int elem) {
+  Layout L{};
+  const int64_t R = T * K;
+  L.B = static_cast<int>((T + moe::kRouterTokensPerCta - 1) / moe::kRouterTokensPerCta);
+  L.Rpad = static_cast<int>(align_up(static_cast<size_t>(R), moe::kTileM));
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 1024);
+    return at;
+  };
+  L.idx32 = take(sizeof(int) * R);
+  L.w32 = take(sizeof(float) * R);
+  L.bcount = take(sizeof(int) * static_cast<size_t>(L.B) * E);
+  L.bbase = take(sizeof(int) * static_cast<size_t>(L.B) * E);
+  L.offsets = take(sizeof(int) * (E + 1));
+  L.perm = take(sizeof(int) * R);
+  L.pos = take(sizeof(int) * R);
+  L.xperm = take(static_cast<size_t>(elem) * L.Rpad * D);
+  L.h = take(static_cast<size_t>(elem) * L.Rpad * F);
+  L.y = take(static_cast<size_t>(elem) * L.Rpad * D);
+  L.total = o;
+  return L;
+}
+
+moe_status_t check_common(int64_t T, int64_t D, int E, int K, moe_dtype_t dt) {
+  if (dt != MOE_F32 && dt != MOE_BF16)
+    return fail(MOE_ERR_DTYPE, "dtype %d not supported (f32 or bf16; float64 is rejected)",
+                static_cast<int>(dt));
+  if (T <= 0 || D <= 0 || E <= 0)
+    return fail(MOE_ERR_INVALID_ARG, "dimensions must be positive (T=%lld D=%lld E=%d)",
+                static_cast<long long>(T), static_cast<long long>(D), E);
+  if (K < 1 || K > E) return fail(MOE_ERR_INVALID_ARG, "top_k=%d outside [1, E=%d]", K, E);
+  if (E > MOE_MAX_EXPERTS)
+    return fail(MOE_ERR_SHAPE, "E=%d exceeds MOE_MAX_EXPERTS=%d", E, MOE_MAX_EXPERTS);
+  if (T * K > INT_MAX - moe::kTileM || T > INT_MAX || D > INT_MAX)
+    return fail(MOE_ERR_SHAPE, "T*K=%lld exceeds the 32-bit row index", static_cast<long long>(T * K));
+  return MOE_OK;
+}
+
+// Row coordinates of the weight matrices are 32-bit in the kernels.
+bool shapes_ok(int64_t T, int64_t D, int64_t F, int E, int K, moe_act_t act) {
+  (void)T;
+  (void)K;
+  const int64_t wrows = static_cast<int64_t>(E) * (act == MOE_ACT_SILU_GATED ? 2 * F : F);
+  return F <= INT_MAX / 2 && wrows + 256 <= INT_MAX && static_cast<int64_t>(E) * D + 256 <= INT_MAX;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_ACT: return "unsupported activation";
+    case MOE_ERR_DTYPE: return "unsupported dtype";
+    case MOE_ERR_SHAPE: return "unsupported shape";
+    case MOE_ERR_ALIGNMENT: return "misaligned pointer or size";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "a bounded wait in a kernel timed out";
+    case MOE_ERR_DEVICE: return "unsupported device";
+  }
+  return "unknown status";
+}
+
+const char* moe_stage_name(int stage) {
+  static const char* names[MOE_NUM_STAGES] = {"router", "permute", "gate_up", "down", "combine"};
+  return (stage >= 0 && stage < MOE_NUM_STAGES) ? names[stage] : "";
+}
+
+size_t moe_ffn_workspace_size(int64_t T, int64_t D, int64_t F, int E, int K, moe_dtype_t dt,
+                              moe_act_t act) {
+  if (check_common(T, D, E, K, dt) != MOE_OK || F <= 0) return 0;
+  if (act != MOE_ACT_SILU_GATED && act != MOE_ACT_RELU) return 0;
+  if (!shapes_ok(T, D, F, E, K, act)) return 0;
+  return layout(T, D, F, E, K, dt == MOE_BF16 ? 2 : 4).total;
+}
+
+moe_status_t moe_route(const void* x, const void* router, const float* router_bias, int64_t T,
+                       int64_t D, int E, int K, int norm_topk_prob, moe_dtype_t dt,
+                       float* router_logits, int64_t* selected_experts, float* routing_weights,
+                       void* stream) {
+  g_last_error.clear();
+  moe_status_t st = check_common(T, D, E, K, dt);
+  if (st != MOE_OK) return st;
+  if (!x || !router || !selected_experts || !routing_weights)
+    return fail(MOE_ERR_INVALID_ARG, "x, router, selected_experts and routing_weights are required");
+  const void* ptrs[] = {x, router, router_bias, router_logits, selected_experts, routing_weights};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(MOE_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+  DevInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != MOE_OK) return st;
+  moe::RouteArgs a{};
+  a.x = x;
+  a.router = router;
+  a.router_bias = router_bias;
+  a.T = static_cast<int>(T);
+  a.D = static_cast<int>(D);
+  a.E = E;
+  a.K = K;
+  a.norm = norm_topk_prob ? 1 : 0;
+  a.dt = dt == MOE_BF16 ? moe::kBF16 : moe::kF32;
+  a.logits = router_logits;
+  a.sel64 = selected_experts;
+  a.wout = routing_weights;
+  cudaError_t e = moe::launch_router(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "router launch");
+  return MOE_OK;
+}
+
+moe_status_t moe_ffn_forward(const void* x, const void* router, const void* gate_up_proj,
+                             const void* down_proj, int E, int K, int norm_topk_prob,
+                             moe_act_t act, void* out, int64_t* selected_experts,
+                             float* routing_weights, int64_t T, int64_t D, int64_t F,
+                             moe_dtype_t dt, const float* router_bias, const float* b1,
+                             const float* b2, float* router_logits, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  moe_status_t st = check_common(T, D, E, K, dt);
+  if (st != MOE_OK) return st;
+  if (act != MOE_ACT_SILU_GATED && act != MOE_ACT_RELU)
+    return fail(MOE_ERR_UNSUPPORTED_ACT, "activation %d not supported (SiLU-gated or ReLU)",
+                static_cast<int>(act));
+  if (F <= 0) return fail(MOE_ERR_INVALID_ARG, "F=%lld must be positive", static_cast<long long>(F));
+  if (!shapes_ok(T, D, F, E, K, act)) return fail(MOE_ERR_SHAPE, "sizes exceed 32-bit indexing");
+  if (!x || !router || !gate_up_proj || !down_proj || !out)
+    return fail(MOE_ERR_INVALID_ARG, "x, router, gate_up_proj, down_proj and out are required");
+  if (act == MOE_ACT_RELU && (!b1 || !b2 || !router_bias))
+    return fail(MOE_ERR_INVALID_ARG, "the ReLU expert needs router_bias, b1 and b2");
+  if (act == MOE_ACT_SILU_GATED && (b1 || b2))
+    return fail(MOE_ERR_INVALID_ARG, "the SiLU-gated expert has no b1/b2");
+  const void* ptrs[] = {x, router, gate_up_proj, down_proj, out, selected_experts, routing_weights,
+                        router_bias, b1, b2, router_logits, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(MOE_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+  if (dt == MOE_BF16 && (D % 8 != 0 || F % 8 != 0))
+    return fail(MOE_ERR_ALIGNMENT, "bf16 path needs D and F multiples of 8 (D=%lld F=%lld)",
+                static_cast<long long>(D), static_cast<long long>(F));
+  const int elem = dt == MOE_BF16 ? 2 : 4;
+  const Layout L = layout(T, D, F, E, K, elem);
+  if (!workspace || workspace_bytes < L.total)
+    return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", L.total,
+                workspace ? workspace_bytes : static_cast<size_t>(0));
+  DevInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != MOE_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* idx32 = reinterpret_cast<int*>(ws + L.idx32);
+  float* w32 = reinterpret_cast<float*>(ws + L.w32);
+  int* bcount = reinterpret_cast<int*>(ws + L.bcount);
+  int* bbase = reinterpret_cast<int*>(ws + L.bbase);
+  int* offsets = reinterpret_cast<int*>(ws + L.offsets);
+  int* perm = reinterpret_cast<int*>(ws + L.perm);
+  int* pos = reinterpret_cast<int*>(ws + L.pos);
+  void* xperm = ws + L.xperm;
+  void* H = ws + L.h;
+  void* Y = ws + L.y;
+  const int Ti = static_cast<int>(T), Di = static_cast<int>(D), Fi = static_cast<int>(F);
+  const int gu_act = act == MOE_ACT_SILU_GATED ? 0 : 1;
+  const int gu_rows = act == MOE_ACT_SILU_GATED ? 2 * Fi : Fi;
+
+  StageTimer timer(s);
+  cudaError_t e = timer.run(0, [&] {
+    moe::RouteArgs a{};
+    a.x = x;
+    a.router = router;
+    a.router_bias = router_bias;
+    a.T = Ti;
+    a.D = Di;
+    a.E = E;
+    a.K = K;
+    a.norm = norm_topk_prob ? 1 : 0;
+    a.dt = dt == MOE_BF16 ? moe::kBF16 : moe::kF32;
+    a.logits = router_logits;
+    a.sel64 = selected_experts;
+    a.wout = routing_weights;
+    a.idx32 = idx32;
+    a.w32 = w32;
+    a.blockcounts = bcount;
+    return moe::launch_router(a, s);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "router launch");
+  e = timer.run(1, [&] {
+    cudaError_t r = moe::launch_permute_scan(bcount, L.B, E, offsets, bbase, s);
+    if (r != cudaSuccess) return r;
+    return moe::launch_permute_scatter(idx32, bbase, Ti, K, E, x, Di, elem, perm, pos, xperm, s);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+  if (dt == MOE_BF16) {
+    e = timer.run(2, [&] {
+      return moe::launch_gemm_tc(gu_act, xperm, L.Rpad, gate_up_proj, offsets, E, Ti, Di, Fi,
+                                 gu_rows, b1, H, dev->err, s);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "gate_up launch");
+    e = timer.run(3, [&] {
+      return moe::launch_gemm_tc(2, H, L.Rpad, down_proj, offsets, E, Ti, Fi, Di, Di, b2, Y,
+                                 dev->err, s);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "down launch");
+  } else {
+    e = timer.run(2, [&] {
+      return moe::launch_gemm_simt_f32(gu_act, static_cast<const float*>(xperm),
+                                       static_cast<const float*>(gate_up_proj), offsets, E, Ti, Di,
+                                       Fi, gu_rows, b1, static_cast<float*>(H), s);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "gate_up launch");
+    e = timer.run(3, [&] {
+      return moe::launch_gemm_simt_f32(2, static_cast<const float*>(H),
+                                       static_cast<const float*>(down_proj), offsets, E, Ti, Fi, Di,
+                                       Di, b2, static_cast<float*>(Y), s);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "down launch");
+  }
+  e = timer.run(4, [&] {
+    return moe::launch_combine(Y, w32, pos, Ti, K, Di, dt == MOE_BF16 ? moe::kBF16 : moe::kF32, out,
+                               s);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  return MOE_OK;
+}
+
+moe_status_t moe_device_status(void* stream) {
+  g_last_error.clear();
+  DevInfo* dev = nullptr;
+  moe_status_t st = device_info(&dev);
+  if (st != MOE_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int word = 0;
+  e = cudaMemcpy(&word, dev->err, sizeof word, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the error word");
+  if (word != 0) {
+    const unsigned int zero = 0;
+    cudaMemcpy(dev->err, &zero, sizeof zero, cudaMemcpyHostToDevice);
+    return fail(MOE_ERR_TIMEOUT, "device error word 0x%x (1 = a bounded wait timed out)", word);
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_profile_enable(int enable) {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  g_prof.enabled = enable != 0;
+  g_prof.recs.clear();
+  g_prof.next = 0;
+  g_prof.calls = 0;
+  return MOE_OK;
+}
+
+int moe_profile_read(float* ms, int n_stages) {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  for (int i = 0; i < n_stages; ++i) ms[i] = 0.f;
+  for (auto& r : g_prof.recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.second.second) == cudaSuccess &&
+        cudaEventElapsedTime(&t, r.second.first, r.second.second) == cudaSuccess &&
+        r.first < n_stages)
+      ms[r.first] += t;
+  }
+  const int calls = g_prof.calls;
+  g_prof.recs.clear();
+  g_prof.next = 0;
+  g_prof.calls = 0;
+  return calls;
+}
+
+}  // extern "C"
+
+namespace moe {
+int num_sms() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  if (dev >= 0 && dev < 64 && g_dev[dev].init) return g_dev[dev].sms;
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 1;
+}
+}  // namespace moe

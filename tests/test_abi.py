@@ -1,0 +1,120 @@
+"""The C ABI on the CPU: the library loads, exports every function the header
+declares, and rejects bad arguments on the host before touching the device.
+
+No call here reaches a kernel: every call fails validation first, which is
+the point (errors are caught before any launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_ffn_09_b200 import moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+P = 0x10000          # a 16-byte aligned stand-in for a device pointer (never dereferenced)
+MIS = 0x10008        # misaligned
+
+
+@pytest.fixture(scope="module")
+def L():
+    from mixture_experts_ffn_09_b200 import build
+    build.build()
+    return moe.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("moe_ffn_forward", "moe_route", "moe_ffn_workspace_size", "moe_status_string",
+              "moe_device_status", "moe_profile_enable", "moe_profile_read"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in declared_functions():
+        assert hasattr(L, n), n
+    out = os.popen(f"nm -D --defined-only {moe.LIB_PATH}").read()
+    exported = set(re.findall(r" T (moe_\w+)", out))
+    assert exported == set(declared_functions())
+
+
+def test_abi_version_and_strings(L):
+    assert moe.abi_version() == 1
+    for s in range(10):
+        assert moe.status_string(s) not in ("", "unknown status")
+    assert moe.status_string(123) == "unknown status"
+
+
+def _fwd(L, **kw):
+    a = dict(x=P, router=P, gu=P, down=P, E=8, K=2, norm=1, act=0, out=P, sel=P, w=P, T=64, D=64,
+             F=128, dt=0, rb=None, b1=None, b2=None, logits=None, ws=P, wsb=1 << 40, stream=None)
+    a.update(kw)
+    return L.moe_ffn_forward(a["x"], a["router"], a["gu"], a["down"], a["E"], a["K"], a["norm"],
+                             a["act"], a["out"], a["sel"], a["w"], a["T"], a["D"], a["F"], a["dt"],
+                             a["rb"], a["b1"], a["b2"], a["logits"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(K=0), moe.MOE_ERR_INVALID_ARG),          # top_k below 1
+    (dict(K=9), moe.MOE_ERR_INVALID_ARG),          # top_k above E
+    (dict(T=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(D=-1), moe.MOE_ERR_INVALID_ARG),
+    (dict(F=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(E=0, K=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(dt=2), moe.MOE_ERR_DTYPE),               # float64 is rejected
+    (dict(dt=7), moe.MOE_ERR_DTYPE),
+    (dict(act=5), moe.MOE_ERR_UNSUPPORTED_ACT),    # anything but SiLU-gated / ReLU
+    (dict(E=300, K=2), moe.MOE_ERR_SHAPE),         # beyond MOE_MAX_EXPERTS
+    (dict(x=None), moe.MOE_ERR_INVALID_ARG),
+    (dict(out=None), moe.MOE_ERR_INVALID_ARG),
+    (dict(act=1), moe.MOE_ERR_INVALID_ARG),        # ReLU without biases
+    (dict(act=0, b1=P, b2=P), moe.MOE_ERR_INVALID_ARG),   # SiLU with biases
+    (dict(x=MIS), moe.MOE_ERR_ALIGNMENT),
+    (dict(dt=1, D=60), moe.MOE_ERR_ALIGNMENT),     # bf16 rows need 16-byte strides
+    (dict(dt=1, F=100), moe.MOE_ERR_ALIGNMENT),
+    (dict(ws=None), moe.MOE_ERR_WORKSPACE),
+    (dict(wsb=16), moe.MOE_ERR_WORKSPACE),
+])
+def test_forward_rejects_on_host(L, kw, code):
+    assert _fwd(L, **kw) == code
+    assert moe.last_error() != ""
+
+
+def test_relu_with_all_biases_passes_validation_up_to_the_device(L):
+    # With every argument valid the call reaches the device query, which
+    # fails on a machine without a GPU (and nothing is launched).
+    import torch
+    st = _fwd(L, act=1, rb=P, b1=P, b2=P)
+    if torch.cuda.is_available():
+        pytest.skip("has a GPU")
+    assert st in (moe.MOE_ERR_CUDA, moe.MOE_ERR_DEVICE)
+
+
+def test_route_rejects_on_host(L):
+    r = lambda **k: L.moe_route(k.get("x", P), P, None, k.get("T", 64), 64, 8, k.get("K", 2), 1,
+                                k.get("dt", 0), None, k.get("sel", P), P, None)
+    assert r(K=0) == moe.MOE_ERR_INVALID_ARG
+    assert r(K=9) == moe.MOE_ERR_INVALID_ARG
+    assert r(T=0) == moe.MOE_ERR_INVALID_ARG
+    assert r(dt=2) == moe.MOE_ERR_DTYPE
+    assert r(sel=None) == moe.MOE_ERR_INVALID_ARG
+    assert r(x=MIS) == moe.MOE_ERR_ALIGNMENT
+
+
+def test_workspace_size(L):
+    ws = moe.workspace_size(64, 64, 128, 8, 2, moe.F32, moe.ACT_SILU_GATED)
+    # 128 routed rows, padded to one 128-row tile: x_perm, H, Y dominate
+    assert ws >= 128 * (64 + 128 + 64) * 4
+    assert ws < 128 * (64 + 128 + 64) * 4 + 64 * 1024
+    assert moe.workspace_size(64, 64, 128, 8, 9, moe.F32) == 0
+    assert moe.workspace_size(64, 64, 128, 8, 2, moe.F64) == 0
+    big = moe.workspace_size(4096, 4096, 14336, 8, 2, moe.BF16)
+    assert big >= 8192 * (4096 + 14336 + 4096) * 2
+    assert big < 8192 * (4096 + 14336 + 4096) * 2 + 8 * 1024 * 1024

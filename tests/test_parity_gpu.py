@@ -1,0 +1,240 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
+the same seeded inputs.  See parity_lib for the comparison rule."""
+import numpy as np
+import pytest
+
+from mixture_experts_ffn_09_b200 import synth
+from oracle import moe_oracle as O
+
+import parity_lib as PL
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from mixture_experts_ffn_09_b200 import build
+    build.build()
+
+
+def _full_check(d, E, K, norm, act, dtype, x_shape=None):
+    """Whole-layer parity on every token (small cases)."""
+    h = PL.host_views(d)
+    dev = PL.to_device(d)
+    g = PL.run_gpu(dev, E, K, norm, act)
+    x = h["x"].reshape(-1, h["x"].shape[-1])
+    r = O.moe_ffn_forward(x, h["router"], h["gate_up_proj"], h["down_proj"], K, norm, act,
+                          h["router_bias"], h["b1"], h["b2"])
+    clear = PL.check_routing(g, r, K, norm)
+    ref = r["out"].copy()
+    if (~clear).any():
+        un = np.nonzero(~clear)[0]
+        ref[un] = PL.oracle_out_for(h, un, g["sel"][un], K, norm, act)
+    PL.check_out(g["out"], ref, dtype)
+    lg_scale = np.abs(r["router_logits"]).max()
+    assert np.abs(g["logits"] - r["router_logits"]).max() <= 1e-5 * max(lg_scale, 1.0)
+    return g, r
+
+
+# ------------------------------------------------------- the five workloads
+def test_dense_relu_exercise_layer():
+    w = synth.DENSE_RELU
+    _full_check(synth.make_inputs(w), w.E, w.K, w.norm_topk_prob, w.act, w.dtype)
+
+
+def test_silu_gated_mojolearn_layer():
+    w = synth.SILU_SMALL
+    d = synth.make_inputs(w)
+    assert d["x"].shape == (4, 16, 64)
+    g, _ = _full_check(d, w.E, w.K, w.norm_topk_prob, w.act, w.dtype)
+
+
+@pytest.fixture(scope="module")
+def decode_case():
+    w = synth.DECODE[1]
+    d = synth.make_inputs(w)
+    h = PL.host_views(d)
+    eo = O.expert_outputs(h["x"], h["gate_up_proj"], h["down_proj"], w.act)   # dense, shared by K
+    return w, d, h, PL.to_device(d), eo
+
+
+@pytest.mark.parametrize("K", [1, 2, 8])
+def test_decode_weight_streaming(decode_case, K):
+    w, d, h, dev, eo = decode_case
+    g = PL.run_gpu(dev, w.E, K, True, w.act)
+    r = O.moe_route(h["x"], h["router"], K, True)
+    clear = PL.check_routing(g, r, K, True)
+    ref = O.combine(eo, r["selected_experts"], r["routing_weights"])
+    if (~clear).any():
+        un = np.nonzero(~clear)[0]
+        v = np.take_along_axis(r["probs"][un], g["sel"][un], 1)
+        ref[un] = O.combine(eo[un], g["sel"][un], O.routing_weights(v, True))
+    PL.check_out(g["out"], ref, "bf16")
+    if K == w.E:
+        # K = E combines every expert: the full softmax-weighted sum
+        full = np.einsum("te,ted->td", r["probs"], eo) / (1 + 1e-9)
+        PL.check_out(g["out"], full, "bf16", "K=E full weighted sum")
+
+
+def _sampled_full_size(w, n_sample):
+    d = synth.make_inputs(w)
+    h = PL.host_views(d)
+    dev = PL.to_device(d)
+    g = PL.run_gpu(dev, w.E, w.K, w.norm_topk_prob, w.act)
+    r = PL.oracle_route(h, w.K, w.norm_topk_prob)
+    clear = PL.check_routing(g, r, w.K, w.norm_topk_prob)
+    assert clear.mean() > 0.99
+    tok = PL.sample_tokens(r["selected_experts"], w.E, n_sample)
+    ref = PL.oracle_out_for(h, tok, g["sel"][tok], w.K, w.norm_topk_prob, w.act)
+    PL.check_out(g["out"][tok], ref, w.dtype)
+    # every token's output is finite and no row was left unwritten
+    assert np.isfinite(g["out"]).all()
+    return g, r
+
+
+def test_mixtral_8x7b_full_size_sampled():
+    _sampled_full_size(synth.MIXTRAL, 48)
+
+
+def test_fine_grained_zipf_full_size_sampled():
+    g, r = _sampled_full_size(synth.FINE_GRAINED, 96)
+    load = np.bincount(g["sel"].ravel(), minlength=64)
+    assert load[0] == load.max()        # the rank-1 expert is the hottest
+
+
+# ------------------------------------------------ shapes, tails, edge cases
+CASES = [
+    # T, D, F, E, K, act, dtype
+    (300, 136, 200, 5, 2, "silu_gated", "bf16"),    # ragged K and N tails
+    (1, 64, 64, 4, 2, "silu_gated", "bf16"),        # one token
+    (257, 128, 256, 8, 8, "silu_gated", "bf16"),    # K = E
+    (130, 72, 88, 3, 1, "silu_gated", "bf16"),      # K = 1
+    (512, 512, 384, 8, 2, "silu_gated", "bf16"),    # several tiles per expert
+    (200, 64, 64, 256, 4, "silu_gated", "bf16"),    # the maximum expert count, most empty
+    (300, 136, 200, 5, 2, "relu", "bf16"),          # biased Dense/ReLU expert on tensor cores
+    (100, 33, 47, 6, 3, "silu_gated", "f32"),       # odd sizes on the fp32 path
+    (77, 50, 30, 4, 2, "relu", "f32"),
+    (1, 8, 8, 1, 1, "silu_gated", "f32"),           # one token, one expert
+    (129, 264, 520, 1, 1, "silu_gated", "bf16"),    # one expert: a plain FFN
+]
+
+
+@pytest.mark.parametrize("T,D,F,E,K,act,dtype", CASES)
+def test_shapes_and_edges(T, D, F, E, K, act, dtype):
+    d = synth.random_case(1000 + T + D + E, T, D, F, E, act=act, dtype=dtype,
+                          weight_std=0.3 if dtype == "f32" else 0.05)
+    _full_check(d, E, K, True, act, dtype)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_norm_topk_prob_off(dtype):
+    d = synth.random_case(7, 96, 64, 64, 6, dtype=dtype, weight_std=0.2)
+    _full_check(d, 6, 3, False, "silu_gated", dtype)
+
+
+def test_all_tokens_to_one_expert():
+    d = dict(synth.random_case(3, 640, 128, 128, 8, dtype="bf16", weight_std=0.05))
+    rb = np.zeros(8, dtype=np.float32)
+    rb[3] = 30.0
+    d["router_bias"] = rb
+    g, _ = _full_check(d, 8, 1, True, "silu_gated", "bf16")
+    assert (g["sel"] == 3).all()
+
+
+def test_tie_break_on_device():
+    """Identical router rows for experts 0 and 1 give identical fp32 logits;
+    the lower index must come first and K=1 never picks expert 1."""
+    d = dict(synth.random_case(5, 256, 64, 64, 4, dtype="bf16", weight_std=0.05))
+    router = d["router"].copy()
+    router[1] = router[0]
+    d["router"] = router
+    g, _ = _full_check(d, 4, 2, True, "silu_gated", "bf16")
+    both = (g["sel"] == 0).any(1) & (g["sel"] == 1).any(1)
+    assert both.any()
+    for row in g["sel"][both]:
+        assert list(row).index(0) < list(row).index(1)
+    g1 = PL.run_gpu(PL.to_device(d), 4, 1, True, "silu_gated")
+    assert not (g1["sel"] == 1).any()
+
+
+def test_worked_example_through_the_device():
+    """The exercise's two-token example run end to end on the device: x
+    picks a column of the router (log-probabilities) and of each expert's
+    linear map (the example's expert outputs)."""
+    import json
+    import os
+    gold = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                       "worked_example_two_tokens.json")))
+    probs = np.array(gold["probs"])
+    eo = np.array(gold["expert_outs"])                   # (T=2, E=3, D=2)
+    x = np.eye(2, dtype=np.float32)                      # token t = e_t
+    router = np.log(probs).T.astype(np.float32)          # logits of token t = log p[t]
+    # ReLU expert with W1 = I, b1 = 0 (h = x >= 0), W2 = [out(x0) out(x1)], b2 = 0
+    W1 = np.stack([np.eye(2, dtype=np.float32)] * 3)
+    W2 = np.stack([eo[:, e, :].T for e in range(3)]).astype(np.float32)
+    d = {"x": x, "router": router, "router_bias": np.zeros(3, np.float32), "gate_up_proj": W1,
+         "down_proj": W2, "b1": np.zeros((3, 2), np.float32), "b2": np.zeros((3, 2), np.float32)}
+    g = PL.run_gpu(PL.to_device(d), 3, 2, True, "relu")
+    assert g["sel"].tolist() == gold["expected_indices"]
+    np.testing.assert_allclose(g["out"], gold["expected_out"], atol=gold["atol"], rtol=0)
+
+
+# ------------------------------------------------------------- properties
+def test_deterministic_bitwise():
+    d = synth.random_case(11, 700, 256, 384, 8, dtype="bf16", weight_std=0.05)
+    dev = PL.to_device(d)
+    a = PL.run_gpu(dev, 8, 2, True, "silu_gated")
+    b = PL.run_gpu(dev, 8, 2, True, "silu_gated")
+    for k in ("out", "sel", "w", "logits"):
+        np.testing.assert_array_equal(a[k], b[k])
+
+
+def test_token_permutation_equivariance_bitwise():
+    d = synth.random_case(12, 500, 256, 256, 8, dtype="bf16", weight_std=0.05)
+    perm = np.random.default_rng(0).permutation(500)
+    d2 = dict(d)
+    d2["x"] = np.ascontiguousarray(d["x"][perm])
+    a = PL.run_gpu(PL.to_device(d), 8, 2, True, "silu_gated")
+    b = PL.run_gpu(PL.to_device(d2), 8, 2, True, "silu_gated")
+    np.testing.assert_array_equal(b["sel"], a["sel"][perm])
+    np.testing.assert_array_equal(b["w"], a["w"][perm])
+    np.testing.assert_array_equal(b["out"], a["out"][perm])
+
+
+# ------------------------------------------------------------- router only
+@pytest.mark.parametrize("name", [synth.SILU_SMALL.name, synth.DENSE_RELU.name])
+def test_route_entry_point(name):
+    import torch
+    from mixture_experts_ffn_09_b200 import moe
+    w = synth.WORKLOADS[name]
+    d = synth.make_inputs(w)
+    h = PL.host_views(d)
+    dev = PL.to_device(d)
+    x = dev["x"].reshape(-1, w.D)
+    sel = torch.empty(w.T, w.K, dtype=torch.int64, device="cuda")
+    wt = torch.empty(w.T, w.K, dtype=torch.float32, device="cuda")
+    lg = torch.empty(w.T, w.E, dtype=torch.float32, device="cuda")
+    moe.route(x, dev["router"], w.K, True, sel, wt, dev["router_bias"], lg)
+    torch.cuda.synchronize()
+    g = {"sel": sel.cpu().numpy(), "w": wt.cpu().numpy().astype(np.float64)}
+    r = PL.oracle_route(h, w.K, True)
+    PL.check_routing(g, r, w.K, True)
+    np.testing.assert_allclose(lg.cpu().numpy(), r["router_logits"], atol=1e-5, rtol=0)
+
+
+def test_binding_rejects_before_launch():
+    import torch
+    from mixture_experts_ffn_09_b200 import moe
+    d = PL.to_device(synth.random_case(1, 16, 64, 64, 4, dtype="bf16"))
+    out = torch.full_like(d["x"], 7.0)
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(moe.MoEError) as ei:
+        moe.ffn_forward(d["x"], d["router"], d["gate_up_proj"], d["down_proj"], 4, 5, True, 0, out,
+                        workspace=ws)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(moe.MoEError) as ei:
+        moe.ffn_forward(d["x"].double(), d["router"].double(), d["gate_up_proj"].double(),
+                        d["down_proj"].double(), 4, 2, True, 0, out.double(), workspace=ws)
+    assert ei.value.status == moe.MOE_ERR_DTYPE
+    torch.cuda.synchronize()
+    assert (out == 7.0).all()     # nothing was launched
