@@ -148,6 +148,40 @@ MOE_API moe_status_t moe_route(const void* x, const void* router, const float* r
                        float* router_logits, int64_t* selected_experts, float* routing_weights,
                        void* stream);
 
+/*
+ * Forward pass that allocates nothing, for callers that cannot obtain device
+ * memory at call time: code running where a device allocation is not
+ * permitted or not available to it, such as a plugin or callback of another
+ * runtime that owns all device memory and hands the plugin only its inputs
+ * and outputs.  The pages have no counterpart; it is an addition of this
+ * library.
+ *
+ * Same arguments and results as moe_ffn_forward, without the workspace:
+ * the scratch lives in one static device array of
+ * MOE_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * this part of the library keeps until the process exits.  Sizes whose
+ * moe_ffn_workspace_size exceeds it are rejected with MOE_ERR_WORKSPACE
+ * before anything is launched (for bf16 that covers e.g. T=32 tokens with
+ * D=4096, F=14336, E=8, K=8).  No cudaMalloc / cudaFree is called.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  All
+ * calls share the one array and it keeps the previous call's contents; no
+ * part of it has to start at zero, since each call writes every scratch
+ * element it later reads (pad rows only feed rows that are never stored).
+ * Calls whose work overlaps on the GPU (e.g. on two streams at once) race
+ * on the array: order them on one stream or with events.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+MOE_API moe_status_t moe_ffn_forward_noalloc(const void* x, const void* router,
+                                             const void* gate_up_proj, const void* down_proj,
+                                             int E, int K, int norm_topk_prob, moe_act_t act,
+                                             void* out, int64_t* selected_experts,
+                                             float* routing_weights, int64_t T, int64_t D,
+                                             int64_t F, moe_dtype_t dt, const float* router_bias,
+                                             const float* b1, const float* b2,
+                                             float* router_logits, void* stream);
+
 /* Short English description of a status code (static storage). */
 MOE_API const char* moe_status_string(moe_status_t status);
 

@@ -59,4 +59,7 @@ cudaError_t launch_gemm_tc(int act, const void* A, int a_rows, const void* W, co
 
 int num_sms();
 
+// Sets the message moe_last_error() returns on this host thread.
+void set_last_error(const char* msg);
+
 }  // namespace moe

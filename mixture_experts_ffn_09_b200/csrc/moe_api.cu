@@ -419,3 +419,7 @@ int num_sms() {
   return n > 0 ? n : 1;
 }
 }  // namespace moe
+
+namespace moe {
+void set_last_error(const char* msg) { g_last_error = msg ? msg : ""; }
+}  // namespace moe

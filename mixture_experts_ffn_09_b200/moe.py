@@ -71,6 +71,9 @@ def lib() -> ctypes.CDLL:
         L.moe_ffn_forward.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, i64, i64, i64,
                                       i32, vp, vp, vp, vp, vp, sz, vp]
         L.moe_ffn_forward.restype = i32
+        L.moe_ffn_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, i64,
+                                              i64, i64, i32, vp, vp, vp, vp, vp]
+        L.moe_ffn_forward_noalloc.restype = i32
         L.moe_route.argtypes = [vp, vp, vp, i64, i64, i32, i32, i32, i32, vp, vp, vp, vp]
         L.moe_route.restype = i32
         L.moe_status_string.argtypes = [i32]
@@ -201,6 +204,43 @@ def ffn_forward(x, router, gate_up_proj, down_proj, E: int, K: int, norm_topk_pr
         _ptr(router_bias), _ptr(b1), _ptr(b2), _ptr(router_logits), _ptr(workspace), ws_bytes,
         _stream(stream))
     _check(st)
+
+
+def ffn_forward_noalloc(x, router, gate_up_proj, down_proj, E: int, K: int, norm_topk_prob: bool,
+                        act, out, selected_experts=None, routing_weights=None, router_bias=None,
+                        b1=None, b2=None, router_logits=None, stream=None) -> None:
+    """moe_ffn_forward_noalloc: the same forward without a workspace, for
+    callers that cannot allocate device memory when they run the layer (the
+    library's static scratch of noalloc_scratch_bytes() is used instead)."""
+    import torch
+    D = int(x.shape[-1])
+    T = int(x.numel() // D) if D else 0
+    F = int(down_proj.shape[-1])
+    dt = _dtype_code(x)
+    a = _act_code(act)
+    if dt in (F32, BF16) and a in (ACT_SILU_GATED, ACT_RELU) and 1 <= K <= E and T > 0:
+        wdt = x.dtype
+        gu_rows = 2 * F if a == ACT_SILU_GATED else F
+        _expect(router, (E, D), "router", wdt)
+        _expect(gate_up_proj, (E, gu_rows, D), "gate_up_proj", wdt)
+        _expect(down_proj, (E, D, F), "down_proj", wdt)
+        _expect(out, tuple(x.shape), "out", wdt)
+        _expect(selected_experts, (T, K), "selected_experts", torch.int64, False)
+        _expect(routing_weights, (T, K), "routing_weights", torch.float32, False)
+        _expect(router_bias, (E,), "router_bias", torch.float32, False)
+        _expect(b1, (E, F), "b1", torch.float32, False)
+        _expect(b2, (E, D), "b2", torch.float32, False)
+        _expect(router_logits, (T, E), "router_logits", torch.float32, False)
+    st = lib().moe_ffn_forward_noalloc(
+        _ptr(x), _ptr(router), _ptr(gate_up_proj), _ptr(down_proj), E, K, int(bool(norm_topk_prob)),
+        a, _ptr(out), _ptr(selected_experts), _ptr(routing_weights), T, D, F, dt,
+        _ptr(router_bias), _ptr(b1), _ptr(b2), _ptr(router_logits), _stream(stream))
+    _check(st)
+
+
+def noalloc_scratch_bytes() -> int:
+    """Size of the static scratch behind ffn_forward_noalloc (32 MiB)."""
+    return 32 << 20
 
 
 def route(x, router, K: int, norm_topk_prob: bool, selected_experts, routing_weights,
