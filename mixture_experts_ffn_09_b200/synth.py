@@ -115,6 +115,13 @@ FINE_GRAINED = _reg(Workload(
     F=1408, E=64, K=6, act=ACT_SILU_GATED, dtype="bf16", norm_topk_prob=True,
     seed=2, x_dist="normal", router_offset="zipf"))
 
+# A Mixtral-shaped layer cut to 2 experts (704 MB of weights, still larger
+# than L2): the size at which a full counter capture of one grouped-GEMM
+# launch stays within a few GB of device memory.
+MIXTRAL_E2 = _reg(Workload(
+    name="mixtral_shape_t2048_d4096_f14336_e2_k2_bf16", T=2048, D=4096, F=14336, E=2, K=2,
+    act=ACT_SILU_GATED, dtype="bf16", norm_topk_prob=True, seed=5, x_dist="normal"))
+
 # Decode-like weight streaming: 32 tokens, swept over top_k.
 DECODE = {k: _reg(Workload(
     name=f"decode_t32_d4096_f14336_e8_k{k}_bf16", T=32, D=4096, F=14336, E=8,
