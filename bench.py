@@ -41,7 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "source": "fallback"}
 NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 L2_BYTES = 126 * 1024 * 1024
-KERNELS_PER_FORWARD = 6   # router, permute scan, permute scatter, gate_up, down, combine
+KERNELS_PER_FORWARD = 7   # router, permute scan, scatter, gather, gate_up, down, combine
 
 
 def load_peaks() -> dict:

@@ -24,20 +24,28 @@ struct RouteArgs {
   int* idx32;               // (T, K) or null
   float* w32;               // (T, K) or null
   int* blockcounts;         // (ceil(T / kRouterTokensPerCta), E) or null
+  unsigned int* err;        // device error word (bounded waits)
 };
 
+// CUDA-core router (any dtype; used for float32).
 cudaError_t launch_router(const RouteArgs& a, cudaStream_t s);
+// Tensor-core router (bf16, E <= 256): same outputs.
+cudaError_t launch_router_tc(const RouteArgs& a, cudaStream_t s);
 
-// Per-expert totals -> offsets (E + 1) and each router block's first row
-// per expert, blockbase (B, E).
-cudaError_t launch_permute_scan(const int* blockcounts, int B, int E, int* offsets,
-                                int* blockbase, cudaStream_t s);
+// Per-expert column scans of the router's 32-token histograms (B, E):
+// blockbase[b, e] = rows of expert e in blocks before b; totals[e].
+cudaError_t launch_permute_scan(const int* blockcounts, int B, int E, int* blockbase,
+                                int* totals, cudaStream_t s);
 
 // Stable scatter of the (token, slot) pairs into expert order: perm[row] =
-// slot, pos[slot] = row, and x_perm[row, :] = x[slot / K, :].
-cudaError_t launch_permute_scatter(const int* idx32, const int* blockbase, int T, int K, int E,
-                                   const void* x, int D, int elem_bytes, int* perm, int* pos,
-                                   void* x_perm, cudaStream_t s);
+// slot, pos[slot] = row; block 0 also writes offsets (E + 1).
+cudaError_t launch_permute_scatter(const int* idx32, const int* blockbase, const int* totals,
+                                   int T, int K, int E, int* offsets, int* perm, int* pos,
+                                   cudaStream_t s);
+
+// x_perm[row, :] = x[perm[row] / K, :] for the R = T*K sorted rows.
+cudaError_t launch_gather_rows(const int* perm, int R, int K, const void* x, int row_bytes,
+                               void* x_perm, cudaStream_t s);
 
 // out[t, :] = sum_k w[t, k] * Y[pos[t, k], :], fp32 sum in k order.
 cudaError_t launch_combine(const void* Y, const float* w32, const int* pos, int T, int K, int D,

@@ -129,7 +129,7 @@ struct StageTimer {
 
 // ------------------------------------------------------ workspace layout
 struct Layout {
-  size_t idx32, w32, bcount, bbase, offsets, perm, pos, xperm, h, y, total;
+  size_t idx32, w32, bcount, bbase, totals, offsets, perm, pos, xperm, h, y, total;
   int B, Rpad;
 };
 
@@ -148,6 +148,7 @@ Layout layout(int64_t T, int64_t D, int64_t F, int E, int K, int elem) {
   L.w32 = take(sizeof(float) * R);
   L.bcount = take(sizeof(int) * static_cast<size_t>(L.B) * E);
   L.bbase = take(sizeof(int) * static_cast<size_t>(L.B) * E);
+  L.totals = take(sizeof(int) * E);
   L.offsets = take(sizeof(int) * (E + 1));
   L.perm = take(sizeof(int) * R);
   L.pos = take(sizeof(int) * R);
@@ -245,7 +246,9 @@ moe_status_t moe_route(const void* x, const void* router, const float* router_bi
   a.logits = router_logits;
   a.sel64 = selected_experts;
   a.wout = routing_weights;
-  cudaError_t e = moe::launch_router(a, static_cast<cudaStream_t>(stream));
+  a.err = dev->err;
+  cudaError_t e = dt == MOE_BF16 ? moe::launch_router_tc(a, static_cast<cudaStream_t>(stream))
+                                 : moe::launch_router(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "router launch");
   return MOE_OK;
 }
@@ -292,6 +295,7 @@ moe_status_t moe_ffn_forward(const void* x, const void* router, const void* gate
   float* w32 = reinterpret_cast<float*>(ws + L.w32);
   int* bcount = reinterpret_cast<int*>(ws + L.bcount);
   int* bbase = reinterpret_cast<int*>(ws + L.bbase);
+  int* totals = reinterpret_cast<int*>(ws + L.totals);
   int* offsets = reinterpret_cast<int*>(ws + L.offsets);
   int* perm = reinterpret_cast<int*>(ws + L.perm);
   int* pos = reinterpret_cast<int*>(ws + L.pos);
@@ -320,13 +324,16 @@ moe_status_t moe_ffn_forward(const void* x, const void* router, const void* gate
     a.idx32 = idx32;
     a.w32 = w32;
     a.blockcounts = bcount;
-    return moe::launch_router(a, s);
+    a.err = dev->err;
+    return dt == MOE_BF16 ? moe::launch_router_tc(a, s) : moe::launch_router(a, s);
   });
   if (e != cudaSuccess) return cuda_fail(e, "router launch");
   e = timer.run(1, [&] {
-    cudaError_t r = moe::launch_permute_scan(bcount, L.B, E, offsets, bbase, s);
+    cudaError_t r = moe::launch_permute_scan(bcount, L.B, E, bbase, totals, s);
     if (r != cudaSuccess) return r;
-    return moe::launch_permute_scatter(idx32, bbase, Ti, K, E, x, Di, elem, perm, pos, xperm, s);
+    r = moe::launch_permute_scatter(idx32, bbase, totals, Ti, K, E, offsets, perm, pos, s);
+    if (r != cudaSuccess) return r;
+    return moe::launch_gather_rows(perm, Ti * K, K, x, Di * elem, xperm, s);
   });
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   if (dt == MOE_BF16) {

@@ -1,0 +1,382 @@
+// bf16 router on the sm_100a tensor cores: logits = x router^T in fp32 via
+// tcgen05.mma (TMA-fed, accumulator in TMEM), then one thread per token
+// reads its row of logits from TMEM and does bias, softmax statistics,
+// top-k and the renormalised weights in registers.
+//
+// Same definitions as the CUDA-core router (router.cu): "Mixture-of-Experts
+// FFN" (crackedaicode.com), "Compute the experts and router" and "Weight the
+// selected outputs"; mojolearn.MoEBlock (router (E, D), lower-index ties,
+// norm_topk_prob).  The logits are a dense (T x D) x (D x E) contraction, so
+// they go to the tensor cores; everything after is per token.
+//
+// CTA = 128 tokens (one MMA tile of M = 128), N = E rounded up to 16..256.
+// warp 0: TMA producer (x tile 128 x 64 and router tile N x 64 per k-block)
+// warp 1: TMEM allocation and the MMA issue
+// warps 2..5: one token per thread (TMEM lane = row).  Each warp also counts
+// the experts chosen by its 32 tokens: the per-32-token histograms the
+// stable permutation uses.
+//
+// Streaming x is latency-bound per SM, so few row tiles (small T) would use
+// few SMs: the D axis is then split over a thread-block cluster of S <= 8
+// CTAs.  Each CTA accumulates its share of D in TMEM and copies the partial
+// logits to its shared memory; after a cluster barrier CTA rank 0 adds the S
+// partials in rank order through distributed shared memory (fixed order:
+// deterministic, no atomics, no global workspace) and runs the per-token
+// epilogue.
+//
+// Top-k without a "taken" set: the k-th choice is the best entry that ranks
+// strictly after the (k-1)-th in the order (value descending, index
+// ascending), so each of the K rounds is one scan over the row.
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int THREADS = 192;
+constexpr int A_BYTES = BM * BK * 2;
+
+template <int NPAD>
+struct Cfg {
+  static constexpr int B_BYTES = NPAD * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (196 * 1024 / STAGE_BYTES) > 12 ? 12 : (196 * 1024 / STAGE_BYTES);
+  static constexpr uint32_t TMEM_COLS = NPAD < 32 ? 32 : NPAD;
+  static constexpr int PART_STRIDE = NPAD + 1;   // padded rows: conflict-free column access
+  static_assert(BM * PART_STRIDE * 4 <= STAGES * STAGE_BYTES, "partials must fit the ring");
+};
+
+struct Params {
+  int T, E, K, norm, num_kb;
+  int S;                  // CTAs per cluster splitting the k-blocks (power of 2, <= num_kb)
+  const float* bias;
+  float* logits;
+  int64_t* sel64;
+  float* wout;
+  int* idx32;
+  float* w32;
+  int* blockcounts;   // (ceil(T/32), E) or null
+  unsigned int* err;
+};
+
+template <int NPAD>
+struct Tail {
+  uint64_t full[Cfg<NPAD>::STAGES];
+  uint64_t empty[Cfg<NPAD>::STAGES];
+  uint64_t tfull;
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+  int hist[4][kMaxExperts];
+};
+
+template <int NPAD>
+constexpr size_t smem_bytes() {
+  return 1024 + Cfg<NPAD>::STAGES * Cfg<NPAD>::STAGE_BYTES + sizeof(Tail<NPAD>);
+}
+
+__device__ __forceinline__ bool ranks_before(float v, int e, float bv, int be) {
+  return v > bv || (v == bv && e < be);
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Reads a float at the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ float ld_dsmem(const float* local, uint32_t rank) {
+  uint32_t a = smem_u32(local), r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(r) : "memory");
+  return v;
+}
+
+template <int NPAD>
+__global__ void __launch_bounds__(THREADS, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const Params p) {
+  using C = Cfg<NPAD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * A_BYTES;
+  Tail<NPAD>* st = reinterpret_cast<Tail<NPAD>*>(smem + C::STAGES * C::STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = p.S > 1 ? cluster_rank() : 0u;
+  const int m0 = (blockIdx.x / p.S) * BM;
+  const int E = p.E;
+  const int kb_lo = static_cast<int>(rank) * p.num_kb / p.S;         // balanced, never empty
+  const int kb_hi = (static_cast<int>(rank) + 1) * p.num_kb / p.S;
+  float* part = reinterpret_cast<float*>(sA);   // reuses the ring once the MMAs are done
+
+  for (int i = threadIdx.x; i < 4 * kMaxExperts; i += THREADS) (&st->hist[0][0])[i] = 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&st->full[s], 1);
+      mbar_init(&st->empty[s], 1);
+    }
+    mbar_init(&st->tfull, 1);
+    mbar_init(&st->mma_done, 1);
+    st->abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&st->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = st->tmem_base;
+  volatile int* abort = &st->abort;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmX);
+      tma_prefetch_desc(&tmW);
+      int stage = 0;
+      uint32_t phase = 0, used = 0, last_parity = 0;
+      for (int kb = kb_lo; kb < kb_hi; ++kb) {
+        if (!mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err)) break;
+        mbar_arrive_expect_tx(&st->full[stage], C::STAGE_BYTES);
+        tma_load_2d(&tmX, &st->full[stage], sA + stage * A_BYTES, kb * BK, m0);
+        tma_load_2d(&tmW, &st->full[stage], sB + stage * C::B_BYTES, kb * BK, 0);
+        used |= 1u << stage;
+        last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+      int dummy = 0;
+      for (int s = 0; s < C::STAGES; ++s)
+        if (used & (1u << s)) mbar_wait(&st->full[s], (last_parity >> s) & 1u, &dummy, p.err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, NPAD);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kb = kb_lo; kb < kb_hi; ++kb) {
+        if (!mbar_wait(&st->full[stage], phase, abort, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
+        const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          umma_bf16(tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
+                    (kb != kb_lo || k != 0) ? 1u : 0u);
+        umma_commit(&st->empty[stage]);
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (ok) umma_commit(&st->tfull);
+      umma_commit(&st->mma_done);
+      int dummy = 0;
+      mbar_wait(&st->mma_done, 0, &dummy, p.err);
+    }
+  } else {
+    // -------------------- partial logits: TMEM -> this CTA's shared memory
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t tb = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    if (mbar_wait(&st->tfull, 0, abort, p.err)) {
+      tc_fence_after();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      for (int c0 = 0; c0 < E; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tb + c0, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c0 + j < NPAD) part[row * C::PART_STRIDE + c0 + j] = __uint_as_float(r[j]);
+      }
+    }
+  }
+  __syncwarp();
+  if (p.S > 1) cluster_sync_all(); else __syncthreads();
+
+  if (warp >= 2 && rank == 0 && !*abort) {
+    // ------------------------------------------------ one token per thread
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const int t = m0 + row;
+    const bool valid = t < p.T;
+    int* hist = st->hist[wq];
+    float* lrow = part + row * C::PART_STRIDE;
+    // sum the split partials in rank order, add the bias, write the logits
+    float m = -INFINITY;
+    for (int e = 0; e < E; ++e) {
+      float v = lrow[e];
+      for (int q = 1; q < p.S; ++q) v += ld_dsmem(lrow + e, static_cast<uint32_t>(q));
+      if (p.bias) v += __ldg(p.bias + e);
+      if (valid && p.logits) p.logits[static_cast<size_t>(t) * E + e] = v;
+      if (isnan(v)) v = -INFINITY;
+      lrow[e] = v;
+      m = fmaxf(m, v);
+    }
+    float s = 0.f;
+    for (int e = 0; e < E; ++e) s += expf(lrow[e] - m);
+    // K rounds of selection
+    float* tmpw = p.w32 ? p.w32 : p.wout;
+    float lv = INFINITY;
+    int le = -1;
+    float psum = 0.f;
+    for (int k = 0; k < p.K; ++k) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+      for (int e = 0; e < E; ++e) {
+        const float v = lrow[e];
+        if (ranks_before(lv, le, v, e) && ranks_before(v, e, bv, be)) {
+          bv = v;
+          be = e;
+        }
+      }
+      lv = bv;
+      le = be;
+      const float pk = expf(bv - m) / s;
+      psum += pk;
+      if (valid) {
+        const size_t o = static_cast<size_t>(t) * p.K + k;
+        tmpw[o] = pk;
+        if (p.sel64) p.sel64[o] = be;
+        if (p.idx32) p.idx32[o] = be;
+        if (p.blockcounts) atomicAdd(&hist[be], 1);
+      }
+    }
+    if (valid) {
+      const float denom = p.norm ? (psum + 1e-9f) : 1.f;
+      for (int k = 0; k < p.K; ++k) {
+        const size_t o = static_cast<size_t>(t) * p.K + k;
+        const float pk = tmpw[o];
+        const float w = p.norm ? pk / denom : pk;
+        if (p.wout) p.wout[o] = w;
+        if (p.w32) p.w32[o] = w;
+      }
+    }
+    if (p.blockcounts) {
+      __syncwarp();
+      const int b = (m0 + wq * 32) / 32;
+      if (m0 + wq * 32 < p.T)
+        for (int e = lane; e < E; e += 32) p.blockcounts[static_cast<size_t>(b) * E + e] = hist[e];
+    }
+  }
+  __syncwarp();
+  // the other CTAs keep their shared memory until rank 0 has read it
+  if (p.S > 1) cluster_sync_all();
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NPAD>
+cudaError_t launch_npad(const RouteArgs& a, cudaStream_t s) {
+  CUtensorMap mx, mw;
+  if (!make_map(&mx, a.x, static_cast<uint64_t>(a.T), static_cast<uint64_t>(a.D), BM) ||
+      !make_map(&mw, a.router, static_cast<uint64_t>(a.E), static_cast<uint64_t>(a.D), NPAD))
+    return cudaErrorInvalidValue;
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64 || !done[dev]) {
+      err = cudaFuncSetAttribute(router_tc_kernel<NPAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem_bytes<NPAD>()));
+      if (err != cudaSuccess) return err;
+      if (dev >= 0 && dev < 64) done[dev] = true;
+    }
+  }
+  Params p;
+  p.T = a.T;
+  p.E = a.E;
+  p.K = a.K;
+  p.norm = a.norm;
+  p.num_kb = (a.D + BK - 1) / BK;
+  p.bias = a.router_bias;
+  p.logits = a.logits;
+  p.sel64 = a.sel64;
+  p.wout = a.wout;
+  p.idx32 = a.idx32;
+  p.w32 = a.w32;
+  p.blockcounts = a.blockcounts;
+  p.err = a.err;
+  const int m_tiles = (a.T + BM - 1) / BM;
+  // split D over a cluster when the row tiles alone would leave SMs idle
+  int S = 1;
+  while (S < 8 && m_tiles * S * 2 <= num_sms() && S * 2 <= p.num_kb) S *= 2;
+  p.S = S;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(m_tiles * p.S);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = smem_bytes<NPAD>();
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.S > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, router_tc_kernel<NPAD>, mx, mw, p);
+}
+
+}  // namespace
+
+cudaError_t launch_router_tc(const RouteArgs& a, cudaStream_t s) {
+  if (a.E <= 16) return launch_npad<16>(a, s);
+  if (a.E <= 32) return launch_npad<32>(a, s);
+  if (a.E <= 64) return launch_npad<64>(a, s);
+  if (a.E <= 128) return launch_npad<128>(a, s);
+  return launch_npad<256>(a, s);
+}
+
+}  // namespace moe
