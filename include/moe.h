@@ -182,6 +182,20 @@ MOE_API moe_status_t moe_ffn_forward_noalloc(const void* x, const void* router,
                                              const float* b1, const float* b2,
                                              float* router_logits, void* stream);
 
+/*
+ * Which tensor-core grouped GEMM the bf16 path uses (process-wide setting):
+ *   MOE_GEMM_AUTO  - CTA pairs when the average expert has >= 512 routed
+ *                    rows (large batches), one CTA per tile otherwise;
+ *   MOE_GEMM_1SM   - always one CTA per 128 x 256 tile;
+ *   MOE_GEMM_2SM   - always CTA pairs (tcgen05 cta_group::2, 256 x 256).
+ * Both give identical results up to fp32 summation order inside the MMA.
+ * Returns the previous mode, or -1 for an unknown mode (nothing changes).
+ */
+#define MOE_GEMM_AUTO 0
+#define MOE_GEMM_1SM 1
+#define MOE_GEMM_2SM 2
+MOE_API int moe_set_gemm_mode(int mode);
+
 /* Short English description of a status code (static storage). */
 MOE_API const char* moe_status_string(moe_status_t status);
 

@@ -1,0 +1,474 @@
+// bf16 grouped GEMM on CTA pairs: tcgen05.mma.cta_group::2, M = 256 rows
+// (128 per CTA) x N = 256, fp32 accumulators in both CTAs' TMEM.
+//
+// Same computation and epilogues as the one-CTA kernel in gemm_tc.cu (the
+// experts of mojolearn.MoEBlock / the Flax exercise, run as one grouped
+// matrix multiplication over the expert-sorted rows; "Mixture of experts",
+// dewml.dev, "Expert computation and placement": fp32 accumulation, one
+// rounding to bf16).  What changes is the operand traffic: each CTA of a
+// pair stages its own 128 rows of A and HALF of the 256 B rows, and the pair's
+// MMA reads both CTAs' shared memory, so a CTA moves 32 KB per k-block for
+// the same 128 x 256 x 64 product that costs 48 KB on one CTA.  The saved
+// shared memory buys a 6-stage ring.
+//
+// Cluster of 2 CTAs (rank 0 = leader), 192 threads each:
+//   warp 0 (both)   TMA producer for this CTA's A rows and B half; the loads
+//                   complete on the LEADER's full barrier, whose expected
+//                   bytes the leader's producer posts for the pair;
+//   warp 1 (both)   allocates 512 TMEM columns for the pair
+//                   (tcgen05.alloc.cta_group::2); in the leader one lane
+//                   issues the pair's MMAs and commits, multicast to both
+//                   CTAs, the stage releases and accumulator completions;
+//   warps 2..5      epilogue of this CTA's 128 rows, as in gemm_tc.cu; each
+//                   warp's release of an accumulator arrives on the
+//                   leader's barrier (8 arrivals per tile).
+// For the gated expert the leader stages the 128 gate rows and the peer the
+// matching 128 up rows, so accumulator columns [0,128) are gate and
+// [128,256) up in both CTAs, exactly as in the one-CTA kernel.
+//
+// A pair tile covers 256 rows of one expert; rows past the expert's end are
+// computed and not stored.  No load uses cluster multicast.
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BMC = 128;                      // rows per CTA
+constexpr int BMP = 256;                      // rows per pair
+constexpr int BK = 64;
+constexpr int BN_MMA = 256;
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BMC * BK * 2;         // 16 KB
+constexpr int B_BYTES = (BN_MMA / 2) * BK * 2;  // 16 KB (this CTA's half)
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+
+enum { kSiluGated = 0, kReluBias = 1, kBias = 2 };
+
+struct Params {
+  const int* offsets;
+  int E;
+  int n_out;
+  int num_kb;
+  int b_rows;
+  int up_off;
+  __nv_bfloat16* out;
+  const float* bias;
+  unsigned int* err;
+};
+
+struct Tail {
+  uint64_t full[STAGES];     // leader: both CTAs' loads of a stage
+  uint64_t empty[STAGES];    // both: the pair's MMAs have read the stage
+  uint64_t tfull[2];         // both: accumulator ready
+  uint64_t tempty[2];        // leader: 8 epilogue warps released the accumulator
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+  int total_tiles;
+  int tile_start[kMaxExperts + 1];
+  int mt[kMaxExperts];
+  int off[kMaxExperts + 1];
+};
+
+constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(Tail);
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on the
+// barrier at `bar_cluster_addr` (the leader's, for a pair).
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_t bar_cluster_addr,
+                                                 void* dst, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrives once on the barrier at this offset in both CTAs of the pair when
+// the pair's MMAs issued so far have completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+
+__device__ __forceinline__ void decode_tile(const Tail* st, int E, int t, int& e, int& m_blk,
+                                            int& n_blk) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (st->tile_start[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  e = lo;
+  const int local = t - st->tile_start[e];
+  const int mt = st->mt[e];
+  n_blk = local / mt;
+  m_blk = local - n_blk * mt;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void store_row32(__nv_bfloat16* rowp, int col0, int n_out,
+                                            const uint32_t (&w)[16]) {
+  uint4* dst = reinterpret_cast<uint4*>(rowp + col0);
+  if (col0 + 32 <= n_out) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (col0 + 8 * q < n_out) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmB, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  Tail* st = reinterpret_cast<Tail*>(smem + STAGES * STAGE_BYTES);
+
+  constexpr int BN_OUT = (EPI == kSiluGated) ? 128 : 256;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int E = p.E;
+  const int n_tiles = (p.n_out + BN_OUT - 1) / BN_OUT;
+  const int cluster_id = blockIdx.x >> 1;
+  const int num_clusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&st->full[s], 1);
+      mbar_init(&st->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&st->tfull[a], 1);
+      mbar_init(&st->tempty[a], 8);
+    }
+    mbar_init(&st->mma_done, 1);
+    st->abort = 0;
+    int acc = 0;
+    for (int e = 0; e < E; ++e) {
+      const int o0 = p.offsets[e], o1 = p.offsets[e + 1];
+      const int mt = (o1 - o0 + BMP - 1) / BMP;
+      st->off[e] = o0;
+      st->mt[e] = mt;
+      st->tile_start[e] = acc;
+      acc += mt * n_tiles;
+    }
+    st->off[E] = p.offsets[E];
+    st->tile_start[E] = acc;
+    st->total_tiles = acc;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&st->tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();     // the leader's barriers exist before the peer signals them
+  tc_fence_after();
+
+  const uint32_t tmem = st->tmem_base;
+  const int total = st->total_tiles;
+  volatile int* abort = &st->abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      int stage = 0;
+      uint32_t phase = 0, used = 0, last_parity = 0;
+      for (int t = cluster_id; t < total && !*abort; t += num_clusters) {
+        int e, m_blk, n_blk;
+        decode_tile(st, E, t, e, m_blk, n_blk);
+        const int rowA = st->off[e] + m_blk * BMP + static_cast<int>(rank) * BMC;
+        const int rowB = (EPI == kSiluGated)
+                             ? e * p.b_rows + n_blk * 128 + (leader ? 0 : p.up_off)
+                             : e * p.b_rows + n_blk * 256 + static_cast<int>(rank) * 128;
+        bool ok = true;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(&st->full[stage], 2 * STAGE_BYTES);
+          const uint32_t fb = map_to_rank(&st->full[stage], 0);
+          tma_load_2d_pair(&tmA, fb, sA + stage * A_BYTES, kb * BK, rowA);
+          tma_load_2d_pair(&tmB, fb, sB + stage * B_BYTES, kb * BK, rowB);
+          used |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      // Let issued loads land before the CTA can leave: the leader sees them
+      // on its full barriers; the peer's complete on the leader's, so the
+      // peer waits for the pair's MMAs to have released its stages.
+      int dummy = 0;
+      for (int s = 0; s < STAGES; ++s)
+        if (used & (1u << s)) {
+          const uint32_t par = (last_parity >> s) & 1u;
+          if (leader) mbar_wait(&st->full[s], par, &dummy, p.err);
+          else mbar_wait(&st->empty[s], par, &dummy, p.err);
+        }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA (leader)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BMP, BN_MMA);
+      int stage = 0;
+      uint32_t phase = 0;
+      int i = 0;
+      for (int t = cluster_id; t < total; t += num_clusters, ++i) {
+        const int acc = i & 1;
+        const uint32_t aph = (i >> 1) & 1;
+        if (!mbar_wait(&st->tempty[acc], aph ^ 1u, abort, p.err)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + acc * BN_MMA;
+        bool ok = true;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&st->full[stage], phase, abort, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_bf16_pair(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
+                           (kb | k) != 0 ? 1u : 0u);
+          umma_commit_pair(&st->empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair(&st->tfull[acc]);
+      }
+      umma_commit_pair(&st->mma_done);
+      int dummy = 0;
+      mbar_wait(&st->mma_done, 0, &dummy, p.err);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int lane_base = (warp & 3) * 32;
+    const uint32_t tempty_leader0 = map_to_rank(&st->tempty[0], 0);
+    const uint32_t tempty_leader1 = map_to_rank(&st->tempty[1], 0);
+    int i = 0;
+    for (int t = cluster_id; t < total; t += num_clusters, ++i) {
+      int e, m_blk, n_blk;
+      decode_tile(st, E, t, e, m_blk, n_blk);
+      const int acc = i & 1;
+      const uint32_t aph = (i >> 1) & 1;
+      if (!mbar_wait(&st->tfull[acc], aph, abort, p.err)) break;
+      tc_fence_after();
+      const int grow = st->off[e] + m_blk * BMP + static_cast<int>(rank) * BMC + lane_base + lane;
+      const bool rvalid = grow < st->off[e + 1];
+      __nv_bfloat16* rowp = p.out + static_cast<size_t>(rvalid ? grow : 0) * p.n_out;
+      const uint32_t tb = tmem + (static_cast<uint32_t>(lane_base) << 16) + acc * BN_MMA;
+      if (EPI == kSiluGated) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tb + c * 32, g);
+          tmem_ld32(tb + 128 + c * 32, u);
+          tmem_ld_wait();
+          const int col0 = n_blk * 128 + c * 32;
+          if (rvalid && col0 < p.n_out) {
+            uint32_t w[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
+              const float u0 = __uint_as_float(u[2 * j]), u1 = __uint_as_float(u[2 * j + 1]);
+              const float h0 = g0 / (1.f + __expf(-g0)) * u0;
+              const float h1 = g1 / (1.f + __expf(-g1)) * u1;
+              w[j] = pack_bf16x2(h0, h1);
+            }
+            store_row32(rowp, col0, p.n_out, w);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tb + c * 32, v);
+          tmem_ld_wait();
+          const int col0 = n_blk * 256 + c * 32;
+          if (rvalid && col0 < p.n_out) {
+            const float* bias = p.bias ? p.bias + static_cast<size_t>(e) * p.n_out + col0 : nullptr;
+            uint32_t w[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              float a0 = __uint_as_float(v[2 * j]), a1 = __uint_as_float(v[2 * j + 1]);
+              if (bias) {
+                if (col0 + 2 * j < p.n_out) a0 += __ldg(bias + 2 * j);
+                if (col0 + 2 * j + 1 < p.n_out) a1 += __ldg(bias + 2 * j + 1);
+              }
+              if (EPI == kReluBias) {
+                a0 = fmaxf(a0, 0.f);
+                a1 = fmaxf(a1, 0.f);
+              }
+              w[j] = pack_bf16x2(a0, a1);
+            }
+            store_row32(rowp, col0, p.n_out, w);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+    }
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  __syncthreads();
+  cluster_sync_all();     // neither CTA frees TMEM while its peer may still use it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), 128u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI>
+cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params& p, int clusters,
+                       cudaStream_t s) {
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64 || !done[dev]) {
+      err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<EPI>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kSmemBytes));
+      if (err != cudaSuccess) return err;
+      if (dev >= 0 && dev < 64) done[dev] = true;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<EPI>, a, b, p);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* W,
+                                const int* offsets, int E, int Kdim, int N, int w_rows_per_expert,
+                                const float* bias, void* C, unsigned int* err, cudaStream_t s) {
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, A, static_cast<uint64_t>(a_rows), static_cast<uint64_t>(Kdim)) ||
+      !make_map(&mb, W, static_cast<uint64_t>(E) * w_rows_per_expert, static_cast<uint64_t>(Kdim)))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.offsets = offsets;
+  p.E = E;
+  p.n_out = N;
+  p.num_kb = (Kdim + BK - 1) / BK;
+  p.b_rows = w_rows_per_expert;
+  p.up_off = (act == kSiluGated) ? N : 0;
+  p.out = static_cast<__nv_bfloat16*>(C);
+  p.bias = bias;
+  p.err = err;
+  const int bn_out = (act == kSiluGated) ? 128 : 256;
+  const long long tiles_bound =
+      (static_cast<long long>(a_rows) / BMP + E) * ((N + bn_out - 1) / bn_out);
+  const int max_clusters = num_sms() / 2;
+  const int clusters = static_cast<int>(tiles_bound < max_clusters ? tiles_bound : max_clusters);
+  if (act == kSiluGated) return launch_epi<kSiluGated>(ma, mb, p, clusters, s);
+  if (act == kReluBias) return launch_epi<kReluBias>(ma, mb, p, clusters, s);
+  return launch_epi<kBias>(ma, mb, p, clusters, s);
+}
+
+}  // namespace moe

@@ -65,6 +65,11 @@ cudaError_t launch_gemm_tc(int act, const void* A, int a_rows, const void* W, co
                            int E, int T, int Kdim, int N, int w_rows_per_expert,
                            const float* bias, void* C, unsigned int* err, cudaStream_t s);
 
+// Same GEMM on CTA pairs (tcgen05 cta_group::2, 256-row tiles).
+cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* W,
+                                const int* offsets, int E, int Kdim, int N, int w_rows_per_expert,
+                                const float* bias, void* C, unsigned int* err, cudaStream_t s);
+
 int num_sms();
 
 // Sets the message moe_last_error() returns on this host thread.

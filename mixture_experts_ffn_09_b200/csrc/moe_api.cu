@@ -12,6 +12,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -22,6 +23,22 @@
 namespace {
 
 thread_local std::string g_last_error;
+
+std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
+
+// The tensor-core GEMM for one launch: CTA pairs pay off when experts have
+// enough rows to fill 256-row tiles.
+cudaError_t launch_gemm_bf16(int act, const void* A, int a_rows, const void* W,
+                             const int* offsets, int E, int T, int K, int Kdim, int N,
+                             int w_rows, const float* bias, void* C, unsigned int* err,
+                             cudaStream_t s) {
+  const int mode = g_gemm_mode.load();
+  const bool pair = mode == MOE_GEMM_2SM ||
+                    (mode == MOE_GEMM_AUTO && static_cast<long long>(T) * K >= 512LL * E);
+  if (pair)
+    return moe::launch_gemm_tc_pair(act, A, a_rows, W, offsets, E, Kdim, N, w_rows, bias, C, err, s);
+  return moe::launch_gemm_tc(act, A, a_rows, W, offsets, E, T, Kdim, N, w_rows, bias, C, err, s);
+}
 
 __device__ unsigned int g_device_error;   // per device: bounded waits that gave up
 
@@ -188,6 +205,11 @@ extern "C" {
 
 int moe_abi_version(void) { return MOE_ABI_VERSION; }
 
+int moe_set_gemm_mode(int mode) {
+  if (mode != MOE_GEMM_AUTO && mode != MOE_GEMM_1SM && mode != MOE_GEMM_2SM) return -1;
+  return g_gemm_mode.exchange(mode);
+}
+
 const char* moe_last_error(void) { return g_last_error.c_str(); }
 
 const char* moe_status_string(moe_status_t s) {
@@ -338,13 +360,13 @@ moe_status_t moe_ffn_forward(const void* x, const void* router, const void* gate
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   if (dt == MOE_BF16) {
     e = timer.run(2, [&] {
-      return moe::launch_gemm_tc(gu_act, xperm, L.Rpad, gate_up_proj, offsets, E, Ti, Di, Fi,
-                                 gu_rows, b1, H, dev->err, s);
+      return launch_gemm_bf16(gu_act, xperm, L.Rpad, gate_up_proj, offsets, E, Ti, K, Di, Fi,
+                              gu_rows, b1, H, dev->err, s);
     });
     if (e != cudaSuccess) return cuda_fail(e, "gate_up launch");
     e = timer.run(3, [&] {
-      return moe::launch_gemm_tc(2, H, L.Rpad, down_proj, offsets, E, Ti, Fi, Di, Di, b2, Y,
-                                 dev->err, s);
+      return launch_gemm_bf16(2, H, L.Rpad, down_proj, offsets, E, Ti, K, Fi, Di, Di, b2, Y,
+                              dev->err, s);
     });
     if (e != cudaSuccess) return cuda_fail(e, "down launch");
   } else {

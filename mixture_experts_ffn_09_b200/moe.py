@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
         L.moe_profile_enable.restype = i32
         L.moe_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), i32]
         L.moe_profile_read.restype = i32
+        L.moe_set_gemm_mode.argtypes = [i32]
+        L.moe_set_gemm_mode.restype = i32
         L.moe_stage_name.argtypes = [i32]
         L.moe_stage_name.restype = ctypes.c_char_p
         _lib = L
@@ -261,6 +263,18 @@ def route(x, router, K: int, norm_topk_prob: bool, selected_experts, routing_wei
                          int(bool(norm_topk_prob)), dt, _ptr(router_logits),
                          _ptr(selected_experts), _ptr(routing_weights), _stream(stream))
     _check(st)
+
+
+GEMM_AUTO, GEMM_1SM, GEMM_2SM = 0, 1, 2
+
+
+def set_gemm_mode(mode: int) -> int:
+    """Selects the bf16 grouped GEMM (GEMM_AUTO, GEMM_1SM, GEMM_2SM);
+    returns the previous mode."""
+    prev = int(lib().moe_set_gemm_mode(int(mode)))
+    if prev < 0:
+        raise ValueError(f"unknown GEMM mode {mode}")
+    return prev
 
 
 def device_status(stream=None) -> int:

@@ -96,6 +96,23 @@ def test_mixtral_8x7b_full_size_sampled():
     _sampled_full_size(synth.MIXTRAL, 48)
 
 
+def test_gemm_variants_agree_on_the_mixtral_layer():
+    """The one-CTA and CTA-pair GEMMs on the full Mixtral-shaped layer: same
+    selection, outputs within the bf16 bound of each other."""
+    from mixture_experts_ffn_09_b200 import moe
+    w = synth.MIXTRAL
+    dev = PL.to_device(synth.make_inputs(w))
+    res = []
+    for mode in (1, 2):
+        prev = moe.set_gemm_mode(mode)
+        try:
+            res.append(PL.run_gpu(dev, w.E, w.K, True, w.act, with_logits=False))
+        finally:
+            moe.set_gemm_mode(prev)
+    np.testing.assert_array_equal(res[0]["sel"], res[1]["sel"])
+    PL.check_out(res[1]["out"], res[0]["out"], "bf16", "pair vs one-CTA GEMM")
+
+
 def test_fine_grained_zipf_full_size_sampled():
     g, r = _sampled_full_size(synth.FINE_GRAINED, 96)
     load = np.bincount(g["sel"].ravel(), minlength=64)
@@ -119,8 +136,22 @@ CASES = [
 ]
 
 
+@pytest.fixture
+def gemm_mode(request):
+    from mixture_experts_ffn_09_b200 import moe
+    prev = moe.set_gemm_mode(request.param)
+    yield request.param
+    moe.set_gemm_mode(prev)
+
+
+MODES = [1, 2]   # one CTA per tile / CTA pairs (the automatic choice is covered by the workloads)
+
+
+@pytest.mark.parametrize("gemm_mode", MODES, indirect=True)
 @pytest.mark.parametrize("T,D,F,E,K,act,dtype", CASES)
-def test_shapes_and_edges(T, D, F, E, K, act, dtype):
+def test_shapes_and_edges(T, D, F, E, K, act, dtype, gemm_mode):
+    if dtype == "f32" and gemm_mode != MODES[0]:
+        pytest.skip("the float32 path has one GEMM")
     d = synth.random_case(1000 + T + D + E, T, D, F, E, act=act, dtype=dtype,
                           weight_std=0.3 if dtype == "f32" else 0.05)
     _full_check(d, E, K, True, act, dtype)
@@ -132,7 +163,8 @@ def test_norm_topk_prob_off(dtype):
     _full_check(d, 6, 3, False, "silu_gated", dtype)
 
 
-def test_all_tokens_to_one_expert():
+@pytest.mark.parametrize("gemm_mode", MODES, indirect=True)
+def test_all_tokens_to_one_expert(gemm_mode):
     d = dict(synth.random_case(3, 640, 128, 128, 8, dtype="bf16", weight_std=0.05))
     rb = np.zeros(8, dtype=np.float32)
     rb[3] = 30.0
@@ -180,7 +212,8 @@ def test_worked_example_through_the_device():
 
 
 # ------------------------------------------------------------- properties
-def test_deterministic_bitwise():
+@pytest.mark.parametrize("gemm_mode", MODES, indirect=True)
+def test_deterministic_bitwise(gemm_mode):
     d = synth.random_case(11, 700, 256, 384, 8, dtype="bf16", weight_std=0.05)
     dev = PL.to_device(d)
     a = PL.run_gpu(dev, 8, 2, True, "silu_gated")
@@ -189,7 +222,8 @@ def test_deterministic_bitwise():
         np.testing.assert_array_equal(a[k], b[k])
 
 
-def test_token_permutation_equivariance_bitwise():
+@pytest.mark.parametrize("gemm_mode", MODES, indirect=True)
+def test_token_permutation_equivariance_bitwise(gemm_mode):
     d = synth.random_case(12, 500, 256, 256, 8, dtype="bf16", weight_std=0.05)
     perm = np.random.default_rng(0).permutation(500)
     d2 = dict(d)
