@@ -33,6 +33,21 @@ Readings where the pages leave a step open (each is listed in the design doc):
   are listed in descending probability (jax.lax.top_k's order, which the
   exercise states).
 
+Routing extensions ("Mixture of experts", dewml.dev, "Router behavior" and
+"Expert computation and placement"; ES-MoE API page, "ESMoE" settings and
+"Balancing objectives"), with the readings the design doc lists:
+
+* sigmoid scores: each expert's score is sigmoid(logit) on its own;
+* a selection bias is added to the scores only to choose the experts; the
+  weights come from the unbiased scores;
+* dynamic_threshold: a kept expert whose renormalised share is below the
+  threshold is dropped, except the first (the leader), and the kept shares
+  are renormalised to sum to one;
+* capacity_factor: each sequence of L tokens keeps
+  floor(max(ceil(L*K/E)*cf, cf)) slots per expert, the first ones in token
+  order; a dropped slot contributes nothing and nothing is renormalised;
+* balancing statistics of a batch from the scores and the dense gate.
+
 Parity status: every function here is pinned by the CPU tests in
 ``tests/test_oracle_pins.py`` (worked example, closed forms, invariants,
 brute force, library special cases).  The pages' own seeded outputs (Flax
@@ -211,6 +226,147 @@ def moe_ffn_given_routing(x, idx, weights, gate_up_proj, down_proj,
     xx = _f64(x).reshape(-1, np.shape(x)[-1])
     eo = expert_outputs(xx, gate_up_proj, down_proj, act, b1, b2)
     return combine(eo, idx, weights)
+
+
+# ------------------------------------------------------ routing extensions
+SCORE_SOFTMAX = "softmax"
+SCORE_SIGMOID = "sigmoid"
+
+
+def sigmoid(z):
+    """sigmoid(z) = 1 / (1 + exp(-z)), one expert at a time ("Mixture of
+    experts", dewml.dev, "Router behavior": softmax or sigmoid scores)."""
+    return 1.0 / (1.0 + np.exp(-_f64(z)))
+
+
+def router_scores(logits, score: str = SCORE_SOFTMAX):
+    if score == SCORE_SOFTMAX:
+        return softmax(logits)
+    if score == SCORE_SIGMOID:
+        return sigmoid(logits)
+    raise NotImplementedError(f"score {score!r}")
+
+
+def select_experts(scores, K: int, selection_bias=None):
+    """Top-K experts by score (+ selection bias), descending, equal values to
+    the lower index.  Returns the chosen indices and their UNBIASED scores
+    (the bias only decides which experts are picked: "Router behavior")."""
+    sc = _f64(scores)
+    rank_by = sc if selection_bias is None else sc + _f64(selection_bias)[None, :]
+    _, idx = top_k(rank_by, K)
+    return np.take_along_axis(sc, idx, axis=-1), idx
+
+
+def apply_dynamic_threshold(weights, threshold: float):
+    """ES-MoE's dynamic_threshold (API page, "ESMoE" settings): a routed
+    expert whose share of the mixture (its weight after the top-k
+    renormalisation) is below the threshold is dropped, the leader (first
+    slot) always stays, and the kept shares are renormalised.  Returns
+    (new weights with zeros at dropped slots, kept mask)."""
+    w = _f64(weights)
+    share = w / w.sum(axis=-1, keepdims=True)
+    keep = share >= threshold
+    keep[:, 0] = True
+    kept = np.where(keep, share, 0.0)
+    return kept / kept.sum(axis=-1, keepdims=True), keep
+
+
+def capacity_slots(length: int, K: int, E: int, capacity_factor: float) -> int:
+    """Slots per expert for one sequence: floor(max(ceil(L*K/E)*cf, cf))
+    ("Expert computation and placement", capacity_factor)."""
+    c = max(int(np.ceil(length * K / E)) * float(capacity_factor), float(capacity_factor))
+    return int(np.floor(c))
+
+
+def capacity_keep(idx, E: int, capacity_factor: float, seq_len: int = 0, active=None):
+    """Which (token, slot) pairs keep their expert under the capacity: per
+    sequence of seq_len tokens (0: the whole batch is one sequence) and per
+    expert, the first capacity_slots(...) pairs in token order.  Slots
+    already inactive (``active`` False) take no capacity."""
+    idx = np.asarray(idx)
+    T, K = idx.shape
+    L = T if not seq_len else int(seq_len)
+    keep = np.zeros((T, K), dtype=bool)
+    act = np.ones((T, K), dtype=bool) if active is None else np.asarray(active, dtype=bool)
+    for s0 in range(0, T, L):
+        s1 = min(T, s0 + L)
+        cap = capacity_slots(s1 - s0, K, E, capacity_factor)
+        used = np.zeros(E, dtype=np.int64)
+        for t in range(s0, s1):
+            for k in range(K):
+                if not act[t, k]:
+                    continue
+                e = idx[t, k]
+                if used[e] < cap:
+                    keep[t, k] = True
+                    used[e] += 1
+    return keep
+
+
+def balance_stats(scores, idx, weights):
+    """The four balancing objectives of ES-MoE's API page ("Balancing
+    objectives") on one batch: probs = the router's scores (T, E), gate =
+    the routing weights scattered to (T, E).
+      switch       = E * sum_i mean(probs)_i * mean(gate > 0)_i
+      gshard       = E * sum_i u_i^2, u = mean(gate) normalised to sum to one
+      master       = (1/E) * sum_i (u_i - 1/E)^2
+      gshard_probs = E * sum_i v_i^2, v = mean(probs) normalised"""
+    p = _f64(scores)
+    T, E = p.shape
+    gate = np.zeros((T, E))
+    np.put_along_axis(gate, np.asarray(idx, dtype=np.int64), _f64(weights), axis=1)
+    mp = p.mean(axis=0)
+    mg = gate.mean(axis=0)
+    frac = (gate > 0).mean(axis=0)
+    u = mg / mg.sum()
+    v = mp / mp.sum()
+    return {"switch": E * float((mp * frac).sum()),
+            "gshard": E * float((u * u).sum()),
+            "master": float(((u - 1.0 / E) ** 2).sum() / E),
+            "gshard_probs": E * float((v * v).sum())}
+
+
+def moe_route_ext(x, router, K: int, norm_topk_prob: bool = True, router_bias=None,
+                  score: str = SCORE_SOFTMAX, selection_bias=None, dynamic_threshold: float = 0.0):
+    """Router with the extensions: scores, biased choice, weights, optional
+    dynamic threshold.  ``active`` marks slots still routed after the
+    threshold."""
+    lg = router_logits(x, router, router_bias)
+    check_top_k(K, lg.shape[-1])
+    sc = router_scores(lg, score)
+    vals, idx = select_experts(sc, K, selection_bias)
+    w = routing_weights(vals, norm_topk_prob)
+    active = np.ones(idx.shape, dtype=bool)
+    if dynamic_threshold and dynamic_threshold > 0:
+        w, active = apply_dynamic_threshold(routing_weights(vals, True), dynamic_threshold)
+    rank_by = sc if selection_bias is None else sc + _f64(selection_bias)[None, :]
+    return {"router_logits": lg, "probs": sc, "selected_experts": idx, "routing_weights": w,
+            "active": active, "gap": topk_gap(rank_by, K)}
+
+
+def moe_ffn_forward_ext(x, router, gate_up_proj, down_proj, K: int, norm_topk_prob: bool = True,
+                        act: str = ACT_SILU_GATED, router_bias=None, b1=None, b2=None,
+                        score: str = SCORE_SOFTMAX, selection_bias=None,
+                        dynamic_threshold: float = 0.0, capacity_factor: float = 0.0,
+                        seq_len: int = 0):
+    """The forward with the routing extensions: slots dropped by the
+    threshold or the capacity contribute nothing."""
+    check_act(act)
+    xx = _f64(x)
+    shape = xx.shape
+    xx = xx.reshape(-1, shape[-1])
+    r = moe_route_ext(xx, router, K, norm_topk_prob, router_bias, score, selection_bias,
+                      dynamic_threshold)
+    keep = r["active"].copy()
+    if capacity_factor and capacity_factor > 0:
+        keep &= capacity_keep(r["selected_experts"], router.shape[0], capacity_factor, seq_len,
+                              r["active"])
+    eo = expert_outputs(xx, gate_up_proj, down_proj, act, b1, b2)
+    out = combine(eo, r["selected_experts"], np.where(keep, r["routing_weights"], 0.0))
+    r["kept"] = keep
+    r["out"] = out.reshape(shape)
+    r["balance"] = balance_stats(r["probs"], r["selected_experts"], r["routing_weights"])
+    return r
 
 
 def parameter_count(E: int, D: int, F: int, act: str = ACT_RELU) -> int:
