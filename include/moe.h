@@ -149,6 +149,71 @@ MOE_API moe_status_t moe_route(const void* x, const void* router, const float* r
                        void* stream);
 
 /*
+ * Routing options (all off when zeroed; a NULL options pointer is the same
+ * as zeroed options, i.e. exactly moe_ffn_forward / moe_route).
+ *
+ *   score             MOE_SCORE_SOFTMAX (default): softmax over the experts;
+ *                     MOE_SCORE_SIGMOID: each expert scored by sigmoid(logit)
+ *                     on its own ("Mixture of experts", dewml.dev, "Router
+ *                     behavior": softmax or sigmoid scores).
+ *   selection_bias    (E) f32 device pointer or NULL: added to the scores
+ *                     only to choose the top-k; the weights come from the
+ *                     unbiased scores (same section: a per-expert bias that
+ *                     changes which experts are picked).
+ *   dynamic_threshold > 0: after the weights, a kept expert whose share of
+ *                     the mixture (renormalised weight) is below the
+ *                     threshold is dropped, the first (leader) always stays,
+ *                     and the kept shares are renormalised to sum to one
+ *                     (ES-MoE API page, "ESMoE" settings, dynamic_threshold).
+ *                     Dropped slots get weight 0 and no expert work.
+ *   capacity_factor   > 0: each sequence of seq_len tokens keeps
+ *                     floor(max(ceil(seq_len*K/E)*cf, cf)) slots per expert,
+ *                     the first in token order; a dropped slot adds nothing
+ *                     and no weight is renormalised ("Expert computation and
+ *                     placement", capacity_factor).  Forward only.
+ *   seq_len           tokens per sequence for the capacity; 0 = the whole
+ *                     batch is one sequence; otherwise a multiple of 32.
+ *   slot_kept         (T, K) u8 device out or NULL: 1 where the slot's
+ *                     expert output enters out, 0 where it was dropped.
+ *   balance           4 f32 device out or NULL: the batch's balancing
+ *                     statistics {switch, gshard, master, gshard_probs}
+ *                     (ES-MoE API page, "Balancing objectives"), from the
+ *                     scores and the final routing weights.  Forward only.
+ *
+ * selected_experts keeps the router's top-k choice even for dropped slots;
+ * routing_weights holds the final weights (0 where the threshold dropped).
+ */
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_t;
+
+typedef struct moe_route_opts {
+  moe_score_t score;
+  const float* selection_bias;
+  float dynamic_threshold;
+  float capacity_factor;
+  int64_t seq_len;
+  uint8_t* slot_kept;
+  float* balance;
+} moe_route_opts_t;
+
+MOE_API moe_status_t moe_ffn_forward_ex(const void* x, const void* router,
+                                        const void* gate_up_proj, const void* down_proj, int E,
+                                        int K, int norm_topk_prob, moe_act_t act, void* out,
+                                        int64_t* selected_experts, float* routing_weights,
+                                        int64_t T, int64_t D, int64_t F, moe_dtype_t dt,
+                                        const float* router_bias, const float* b1,
+                                        const float* b2, float* router_logits, void* workspace,
+                                        size_t workspace_bytes, const moe_route_opts_t* opts,
+                                        void* stream);
+
+/* Router only with options (capacity_factor and balance need the forward:
+ * MOE_ERR_INVALID_ARG here). */
+MOE_API moe_status_t moe_route_ex(const void* x, const void* router, const float* router_bias,
+                                  int64_t T, int64_t D, int E, int K, int norm_topk_prob,
+                                  moe_dtype_t dt, float* router_logits, int64_t* selected_experts,
+                                  float* routing_weights, const moe_route_opts_t* opts,
+                                  void* stream);
+
+/*
  * Forward pass that allocates nothing, for callers that cannot obtain device
  * memory at call time: code running where a device allocation is not
  * permitted or not available to it, such as a plugin or callback of another

@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(kThreads) combine_bf16_kernel(const __nv_bfloa
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     for (int k = 0; k < K; ++k) {
+      if (sp[k] < 0) continue;                 // a dropped slot adds nothing
       float y[8];
       load8(Y + static_cast<size_t>(sp[k]) * D + d, y);
       const float wk = sw[k];
@@ -73,7 +74,8 @@ __global__ void __launch_bounds__(kThreads) combine_f32_kernel(const float* __re
   __syncthreads();
   for (int d = threadIdx.x; d < D; d += kThreads) {
     float acc = 0.f;
-    for (int k = 0; k < K; ++k) acc = fmaf(sw[k], __ldg(Y + static_cast<size_t>(sp[k]) * D + d), acc);
+    for (int k = 0; k < K; ++k)
+      if (sp[k] >= 0) acc = fmaf(sw[k], __ldg(Y + static_cast<size_t>(sp[k]) * D + d), acc);
     out[static_cast<size_t>(t) * D + d] = acc;
   }
 }

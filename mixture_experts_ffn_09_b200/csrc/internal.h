@@ -25,7 +25,29 @@ struct RouteArgs {
   float* w32;               // (T, K) or null
   int* blockcounts;         // (ceil(T / kRouterTokensPerCta), E) or null
   unsigned int* err;        // device error word (bounded waits)
+  // routing extensions (all off when zero / null)
+  int score;                // 0: softmax over experts, 1: sigmoid per expert
+  const float* sel_bias;    // (E): added to the scores only to choose the experts
+  float dyn_threshold;      // > 0: drop kept experts whose renormalised share is below it
+  uint8_t* slot_kept;       // (T, K): 1 where the slot's expert output enters out
+  float* bal_partial;       // (parts, 3, E): per-CTA sums of scores, gate, gate > 0
 };
+
+// Slots the router dropped carry this expert index in idx32 (= E).
+// Parts of the balance partials each router flavour writes.
+int router_tc_parts(int T);
+int router_simt_parts(int T);
+
+// Balancing statistics {switch, gshard, master, gshard_probs} from the
+// router's partial sums, in fixed order.
+cudaError_t launch_balance_finalize(const float* partial, int parts, int E, int T, float* out4,
+                                    cudaStream_t s);
+
+// Capacity: clamps the 32-token block histograms in place so that each
+// sequence keeps at most floor(max(ceil(L*K/E)*cf, cf)) slots per expert,
+// the first in token order.  L is a multiple of 32 (0: one sequence).
+cudaError_t launch_capacity_clamp(int* blockcounts, int B, int E, int T, int K, int seq_len,
+                                  float capacity_factor, cudaStream_t s);
 
 // CUDA-core router (any dtype; used for float32).
 cudaError_t launch_router(const RouteArgs& a, cudaStream_t s);
@@ -39,15 +61,19 @@ cudaError_t launch_permute_scan(const int* blockcounts, int B, int E, int* block
 
 // Stable scatter of the (token, slot) pairs into expert order: perm[row] =
 // slot, pos[slot] = row; block 0 also writes offsets (E + 1).
+// Slots whose in-block rank reaches the (clamped) block count, and slots
+// with the sentinel expert, get no row: pos = -1, slot_kept = 0.
 cudaError_t launch_permute_scatter(const int* idx32, const int* blockbase, const int* totals,
-                                   int T, int K, int E, int* offsets, int* perm, int* pos,
-                                   cudaStream_t s);
+                                   const int* blockcounts, int T, int K, int E, int* offsets,
+                                   int* perm, int* pos, uint8_t* slot_kept, cudaStream_t s);
 
-// x_perm[row, :] = x[perm[row] / K, :] for the R = T*K sorted rows.
-cudaError_t launch_gather_rows(const int* perm, int R, int K, const void* x, int row_bytes,
-                               void* x_perm, cudaStream_t s);
+// x_perm[row, :] = x[perm[row] / K, :] for the sorted rows (at most
+// R_max = T*K; the live count is offsets[E]).
+cudaError_t launch_gather_rows(const int* perm, const int* offsets, int E, int R_max, int K,
+                               const void* x, int row_bytes, void* x_perm, cudaStream_t s);
 
-// out[t, :] = sum_k w[t, k] * Y[pos[t, k], :], fp32 sum in k order.
+// out[t, :] = sum_k w[t, k] * Y[pos[t, k], :], fp32 sum in k order; slots
+// with pos < 0 (dropped) add nothing.
 cudaError_t launch_combine(const void* Y, const float* w32, const int* pos, int T, int K, int D,
                            int dt, void* out, cudaStream_t s);
 

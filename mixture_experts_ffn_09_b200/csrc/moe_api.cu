@@ -146,7 +146,7 @@ struct StageTimer {
 
 // ------------------------------------------------------ workspace layout
 struct Layout {
-  size_t idx32, w32, bcount, bbase, totals, offsets, perm, pos, xperm, h, y, total;
+  size_t idx32, w32, bcount, bbase, totals, offsets, perm, pos, bal, xperm, h, y, total;
   int B, Rpad;
 };
 
@@ -169,6 +169,12 @@ Layout layout(int64_t T, int64_t D, int64_t F, int E, int K, int elem) {
   L.offsets = take(sizeof(int) * (E + 1));
   L.perm = take(sizeof(int) * R);
   L.pos = take(sizeof(int) * R);
+  {
+    const int parts = moe::router_simt_parts(static_cast<int>(T)) > moe::router_tc_parts(static_cast<int>(T))
+                          ? moe::router_simt_parts(static_cast<int>(T))
+                          : moe::router_tc_parts(static_cast<int>(T));
+    L.bal = take(sizeof(float) * 3 * static_cast<size_t>(parts) * E);
+  }
   L.xperm = take(static_cast<size_t>(elem) * L.Rpad * D);
   L.h = take(static_cast<size_t>(elem) * L.Rpad * F);
   L.y = take(static_cast<size_t>(elem) * L.Rpad * D);
@@ -197,6 +203,33 @@ bool shapes_ok(int64_t T, int64_t D, int64_t F, int E, int K, moe_act_t act) {
   (void)K;
   const int64_t wrows = static_cast<int64_t>(E) * (act == MOE_ACT_SILU_GATED ? 2 * F : F);
   return F <= INT_MAX / 2 && wrows + 256 <= INT_MAX && static_cast<int64_t>(E) * D + 256 <= INT_MAX;
+}
+
+moe_status_t check_opts(const moe_route_opts_t* o, bool forward) {
+  if (!o) return MOE_OK;
+  if (o->score != MOE_SCORE_SOFTMAX && o->score != MOE_SCORE_SIGMOID)
+    return fail(MOE_ERR_INVALID_ARG, "unknown score function %d", static_cast<int>(o->score));
+  if (!(o->dynamic_threshold >= 0.f) || !(o->capacity_factor >= 0.f) ||
+      !(o->dynamic_threshold < 1e30f) || !(o->capacity_factor < 1e30f))
+    return fail(MOE_ERR_INVALID_ARG, "dynamic_threshold and capacity_factor must be finite and >= 0");
+  if (o->seq_len < 0 || (o->seq_len > 0 && o->seq_len % moe::kRouterTokensPerCta != 0))
+    return fail(MOE_ERR_INVALID_ARG, "seq_len must be 0 or a multiple of %d (got %lld)",
+                moe::kRouterTokensPerCta, static_cast<long long>(o->seq_len));
+  if (!forward && (o->capacity_factor > 0.f || o->balance))
+    return fail(MOE_ERR_INVALID_ARG, "capacity_factor and balance need moe_ffn_forward_ex");
+  if (o->selection_bias && !aligned16(o->selection_bias))
+    return fail(MOE_ERR_ALIGNMENT, "selection_bias must be 16-byte aligned");
+  if (o->balance && (reinterpret_cast<uintptr_t>(o->balance) & 3u))
+    return fail(MOE_ERR_ALIGNMENT, "balance must be 4-byte aligned");
+  return MOE_OK;
+}
+
+void apply_opts(moe::RouteArgs& a, const moe_route_opts_t* o) {
+  if (!o) return;
+  a.score = o->score == MOE_SCORE_SIGMOID ? 1 : 0;
+  a.sel_bias = o->selection_bias;
+  a.dyn_threshold = o->dynamic_threshold;
+  a.slot_kept = o->slot_kept;
 }
 
 }  // namespace
@@ -245,9 +278,18 @@ moe_status_t moe_route(const void* x, const void* router, const float* router_bi
                        int64_t D, int E, int K, int norm_topk_prob, moe_dtype_t dt,
                        float* router_logits, int64_t* selected_experts, float* routing_weights,
                        void* stream) {
+  return moe_route_ex(x, router, router_bias, T, D, E, K, norm_topk_prob, dt, router_logits,
+                      selected_experts, routing_weights, nullptr, stream);
+}
+
+moe_status_t moe_route_ex(const void* x, const void* router, const float* router_bias, int64_t T,
+                          int64_t D, int E, int K, int norm_topk_prob, moe_dtype_t dt,
+                          float* router_logits, int64_t* selected_experts, float* routing_weights,
+                          const moe_route_opts_t* opts, void* stream) {
   g_last_error.clear();
   moe_status_t st = check_common(T, D, E, K, dt);
   if (st != MOE_OK) return st;
+  if ((st = check_opts(opts, false)) != MOE_OK) return st;
   if (!x || !router || !selected_experts || !routing_weights)
     return fail(MOE_ERR_INVALID_ARG, "x, router, selected_experts and routing_weights are required");
   const void* ptrs[] = {x, router, router_bias, router_logits, selected_experts, routing_weights};
@@ -269,6 +311,7 @@ moe_status_t moe_route(const void* x, const void* router, const float* router_bi
   a.sel64 = selected_experts;
   a.wout = routing_weights;
   a.err = dev->err;
+  apply_opts(a, opts);
   cudaError_t e = dt == MOE_BF16 ? moe::launch_router_tc(a, static_cast<cudaStream_t>(stream))
                                  : moe::launch_router(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "router launch");
@@ -282,9 +325,23 @@ moe_status_t moe_ffn_forward(const void* x, const void* router, const void* gate
                              moe_dtype_t dt, const float* router_bias, const float* b1,
                              const float* b2, float* router_logits, void* workspace,
                              size_t workspace_bytes, void* stream) {
+  return moe_ffn_forward_ex(x, router, gate_up_proj, down_proj, E, K, norm_topk_prob, act, out,
+                            selected_experts, routing_weights, T, D, F, dt, router_bias, b1, b2,
+                            router_logits, workspace, workspace_bytes, nullptr, stream);
+}
+
+moe_status_t moe_ffn_forward_ex(const void* x, const void* router, const void* gate_up_proj,
+                                const void* down_proj, int E, int K, int norm_topk_prob,
+                                moe_act_t act, void* out, int64_t* selected_experts,
+                                float* routing_weights, int64_t T, int64_t D, int64_t F,
+                                moe_dtype_t dt, const float* router_bias, const float* b1,
+                                const float* b2, float* router_logits, void* workspace,
+                                size_t workspace_bytes, const moe_route_opts_t* opts,
+                                void* stream) {
   g_last_error.clear();
   moe_status_t st = check_common(T, D, E, K, dt);
   if (st != MOE_OK) return st;
+  if ((st = check_opts(opts, true)) != MOE_OK) return st;
   if (act != MOE_ACT_SILU_GATED && act != MOE_ACT_RELU)
     return fail(MOE_ERR_UNSUPPORTED_ACT, "activation %d not supported (SiLU-gated or ReLU)",
                 static_cast<int>(act));
@@ -324,6 +381,11 @@ moe_status_t moe_ffn_forward(const void* x, const void* router, const void* gate
   void* xperm = ws + L.xperm;
   void* H = ws + L.h;
   void* Y = ws + L.y;
+  float* bal = reinterpret_cast<float*>(ws + L.bal);
+  const float cap = opts ? opts->capacity_factor : 0.f;
+  const int seq_len = opts ? static_cast<int>(opts->seq_len) : 0;
+  float* balance_out = opts ? opts->balance : nullptr;
+  uint8_t* slot_kept = opts ? opts->slot_kept : nullptr;
   const int Ti = static_cast<int>(T), Di = static_cast<int>(D), Fi = static_cast<int>(F);
   const int gu_act = act == MOE_ACT_SILU_GATED ? 0 : 1;
   const int gu_rows = act == MOE_ACT_SILU_GATED ? 2 * Fi : Fi;
@@ -347,15 +409,26 @@ moe_status_t moe_ffn_forward(const void* x, const void* router, const void* gate
     a.w32 = w32;
     a.blockcounts = bcount;
     a.err = dev->err;
-    return dt == MOE_BF16 ? moe::launch_router_tc(a, s) : moe::launch_router(a, s);
+    apply_opts(a, opts);
+    a.bal_partial = balance_out ? bal : nullptr;
+    cudaError_t r = dt == MOE_BF16 ? moe::launch_router_tc(a, s) : moe::launch_router(a, s);
+    if (r != cudaSuccess || !balance_out) return r;
+    const int parts = dt == MOE_BF16 ? moe::router_tc_parts(Ti) : moe::router_simt_parts(Ti);
+    return moe::launch_balance_finalize(bal, parts, E, Ti, balance_out, s);
   });
   if (e != cudaSuccess) return cuda_fail(e, "router launch");
   e = timer.run(1, [&] {
-    cudaError_t r = moe::launch_permute_scan(bcount, L.B, E, bbase, totals, s);
+    cudaError_t r = cudaSuccess;
+    if (cap > 0.f) {
+      r = moe::launch_capacity_clamp(bcount, L.B, E, Ti, K, seq_len, cap, s);
+      if (r != cudaSuccess) return r;
+    }
+    r = moe::launch_permute_scan(bcount, L.B, E, bbase, totals, s);
     if (r != cudaSuccess) return r;
-    r = moe::launch_permute_scatter(idx32, bbase, totals, Ti, K, E, offsets, perm, pos, s);
+    r = moe::launch_permute_scatter(idx32, bbase, totals, bcount, Ti, K, E, offsets, perm, pos,
+                                    slot_kept, s);
     if (r != cudaSuccess) return r;
-    return moe::launch_gather_rows(perm, Ti * K, K, x, Di * elem, xperm, s);
+    return moe::launch_gather_rows(perm, offsets, E, Ti * K, K, x, Di * elem, xperm, s);
   });
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   if (dt == MOE_BF16) {

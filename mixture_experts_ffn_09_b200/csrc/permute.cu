@@ -10,6 +10,7 @@
 //             and the expert's total;
 //   scatter - one CTA per 32-token block ranks its slots within their
 //             expert (warp match + per-warp counts) and writes perm / pos;
+//             slots the router dropped, or past a capacity, get no row;
 //   gather  - one warp per sorted row copies the token row into x_perm.
 #include "common.cuh"
 #include "internal.h"
@@ -59,10 +60,17 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(const int* _
 constexpr int kScatterThreads = 256;
 constexpr int kScatterWarps = kScatterThreads / 32;
 
+// One CTA per 32-token block.  A slot's row is its expert's offset + the
+// rows of that expert in earlier blocks + its rank among the block's slots
+// of the same expert (token order).  When the block counts were clamped by
+// a capacity, slots ranked at or past the clamped count get no row.
 __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
     const int* __restrict__ idx32, const int* __restrict__ blockbase, const int* __restrict__ totals,
-    int T, int K, int E, int* __restrict__ offsets, int* __restrict__ perm, int* __restrict__ pos) {
+    const int* __restrict__ blockcounts, int T, int K, int E, int* __restrict__ offsets,
+    int* __restrict__ perm, int* __restrict__ pos, uint8_t* __restrict__ slot_kept) {
   __shared__ int off[kMaxExperts + 1];
+  __shared__ int base[kMaxExperts];
+  __shared__ int kept[kMaxExperts];
   __shared__ int run[kMaxExperts];
   __shared__ int wc[kScatterWarps][kMaxExperts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -79,7 +87,9 @@ __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
   if (b == 0)
     for (int e = threadIdx.x; e <= E; e += kScatterThreads) offsets[e] = off[e];
   for (int e = threadIdx.x; e < E; e += kScatterThreads) {
-    run[e] = off[e] + blockbase[static_cast<size_t>(b) * E + e];
+    base[e] = off[e] + blockbase[static_cast<size_t>(b) * E + e];
+    kept[e] = blockcounts[static_cast<size_t>(b) * E + e];
+    run[e] = 0;
 #pragma unroll
     for (int w = 0; w < kScatterWarps; ++w) wc[w][e] = 0;
   }
@@ -91,17 +101,29 @@ __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
 
   for (int c0 = s_lo; c0 < s_hi; c0 += kScatterThreads) {
     const int s = c0 + threadIdx.x;
-    const bool valid = s < s_hi;
-    const int e = valid ? idx32[s] : -1;
+    const bool in_range = s < s_hi;
+    int e = in_range ? idx32[s] : -1;
+    if (e >= E) e = -1;                       // dropped by the router: no row, no rank
     const unsigned int mask = __match_any_sync(0xffffffffu, e);
     const int wrank = __popc(mask & lanemask_lt());
-    if (valid && lane == __ffs(mask) - 1) wc[warp][e] = __popc(mask);
+    if (e >= 0 && lane == __ffs(mask) - 1) wc[warp][e] = __popc(mask);
     __syncthreads();
-    if (valid) {
-      int r = run[e] + wrank;
-      for (int w = 0; w < warp; ++w) r += wc[w][e];
-      perm[r] = s;
-      pos[s] = r;
+    if (in_range) {
+      bool has_row = false;
+      if (e >= 0) {
+        int q = run[e] + wrank;
+        for (int w = 0; w < warp; ++w) q += wc[w][e];
+        if (q < kept[e]) {
+          const int r = base[e] + q;
+          perm[r] = s;
+          pos[s] = r;
+          has_row = true;
+        }
+      }
+      if (!has_row) {
+        pos[s] = -1;
+        if (slot_kept) slot_kept[s] = 0;
+      }
     }
     __syncthreads();
     for (int ee = threadIdx.x; ee < E; ee += kScatterThreads) {
@@ -120,13 +142,14 @@ __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
 constexpr int kGatherThreads = 256;
 
 __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const int* __restrict__ perm,
-                                                                     int R, int K,
+                                                                     const int* __restrict__ offsets,
+                                                                     int E, int K,
                                                                      const uint8_t* __restrict__ x,
                                                                      int row_bytes,
                                                                      uint8_t* __restrict__ x_perm) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * (kGatherThreads / 32) + warp;
-  if (r >= R) return;
+  if (r >= offsets[E]) return;
   const int t = perm[r] / K;
   const uint8_t* src = x + static_cast<size_t>(t) * row_bytes;
   uint8_t* dst = x_perm + static_cast<size_t>(r) * row_bytes;
@@ -148,20 +171,22 @@ cudaError_t launch_permute_scan(const int* blockcounts, int B, int E, int* block
   return cudaGetLastError();
 }
 
-cudaError_t launch_permute_scatter(const int* idx32, const int* blockbase, const int* totals, int T,
-                                   int K, int E, int* offsets, int* perm, int* pos, cudaStream_t s) {
+cudaError_t launch_permute_scatter(const int* idx32, const int* blockbase, const int* totals,
+                                   const int* blockcounts, int T, int K, int E, int* offsets,
+                                   int* perm, int* pos, uint8_t* slot_kept, cudaStream_t s) {
   const int B = (T + kRouterTokensPerCta - 1) / kRouterTokensPerCta;
-  permute_scatter_kernel<<<B, kScatterThreads, 0, s>>>(idx32, blockbase, totals, T, K, E, offsets,
-                                                        perm, pos);
+  permute_scatter_kernel<<<B, kScatterThreads, 0, s>>>(idx32, blockbase, totals, blockcounts, T, K,
+                                                        E, offsets, perm, pos, slot_kept);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather_rows(const int* perm, int R, int K, const void* x, int row_bytes,
-                               void* x_perm, cudaStream_t s) {
+cudaError_t launch_gather_rows(const int* perm, const int* offsets, int E, int R_max, int K,
+                               const void* x, int row_bytes, void* x_perm, cudaStream_t s) {
   const int rows_per_cta = kGatherThreads / 32;
-  const int grid = (R + rows_per_cta - 1) / rows_per_cta;
-  gather_rows_kernel<<<grid, kGatherThreads, 0, s>>>(perm, R, K, static_cast<const uint8_t*>(x),
-                                                     row_bytes, static_cast<uint8_t*>(x_perm));
+  const int grid = (R_max + rows_per_cta - 1) / rows_per_cta;
+  gather_rows_kernel<<<grid, kGatherThreads, 0, s>>>(perm, offsets, E, K,
+                                                     static_cast<const uint8_t*>(x), row_bytes,
+                                                     static_cast<uint8_t*>(x_perm));
   return cudaGetLastError();
 }
 

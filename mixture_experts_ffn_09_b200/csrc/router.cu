@@ -15,6 +15,8 @@
 // monotone), so ties in the logits are ties in the probabilities.
 #include <math.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -65,9 +67,12 @@ __global__ void __launch_bounds__(kWarps * 32) router_topk_kernel(RouteArgs a) {
   float* lg_all = sm + E;                                      // kWarps * E
   int* sel_all = reinterpret_cast<int*>(lg_all + kWarps * E);  // kWarps * K
   float* selv_all = reinterpret_cast<float*>(sel_all + kWarps * K);
+  float* bal_all = selv_all + kWarps * K;                      // kWarps * 3 * E (balance only)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  if (a.bal_partial)
+    for (int i = threadIdx.x; i < kWarps * 3 * E; i += blockDim.x) bal_all[i] = 0.f;
   __syncthreads();
 
   const Tin* X = static_cast<const Tin*>(a.x);
@@ -75,6 +80,7 @@ __global__ void __launch_bounds__(kWarps * 32) router_topk_kernel(RouteArgs a) {
   float* lg = lg_all + warp * E;
   int* sel = sel_all + warp * K;
   float* selv = selv_all + warp * K;
+  float* bal = bal_all + warp * 3 * E;
 
   for (int j = 0; j < kRouterTokensPerCta / kWarps; ++j) {
     const int t = blockIdx.x * kRouterTokensPerCta + j * kWarps + warp;
@@ -120,8 +126,8 @@ __global__ void __launch_bounds__(kWarps * 32) router_topk_kernel(RouteArgs a) {
     }
     __syncwarp();
 
-    // ---- bias, logits out, softmax statistics
-    float l[kPerLane];
+    // ---- bias, logits out, softmax statistics, scores and ranking keys
+    float l[kPerLane], sc[kPerLane], key[kPerLane];
     float m = -INFINITY;
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) {
@@ -137,10 +143,23 @@ __global__ void __launch_bounds__(kWarps * 32) router_topk_kernel(RouteArgs a) {
     }
     m = warp_max(m);
     float s = 0.f;
+    if (a.score == 0) {
 #pragma unroll
-    for (int i = 0; i < kPerLane; ++i)
-      if (lane + 32 * i < E) s += expf(l[i] - m);
-    s = warp_sum(s);
+      for (int i = 0; i < kPerLane; ++i)
+        if (lane + 32 * i < E) s += expf(l[i] - m);
+      s = warp_sum(s);
+    }
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) {
+      const int e = lane + 32 * i;
+      sc[i] = 0.f;
+      key[i] = -INFINITY;
+      if (e < E) {
+        sc[i] = a.score == 0 ? expf(l[i] - m) / s : 1.f / (1.f + expf(-l[i]));
+        key[i] = a.sel_bias ? sc[i] + __ldg(a.sel_bias + e) : l[i];
+        if (a.bal_partial) bal[e] += sc[i];
+      }
+    }
 
     // ---- top-k: K rounds of a warp-wide argmax over the untaken experts
     unsigned int taken = 0u;
@@ -150,8 +169,8 @@ __global__ void __launch_bounds__(kWarps * 32) router_topk_kernel(RouteArgs a) {
 #pragma unroll
       for (int i = 0; i < kPerLane; ++i) {
         const int e = lane + 32 * i;
-        if (e < E && !(taken & (1u << i)) && ranks_before(l[i], e, bv, be)) {
-          bv = l[i];
+        if (e < E && !(taken & (1u << i)) && ranks_before(key[i], e, bv, be)) {
+          bv = key[i];
           be = e;
         }
       }
@@ -164,49 +183,94 @@ __global__ void __launch_bounds__(kWarps * 32) router_topk_kernel(RouteArgs a) {
           be = oe;
         }
       }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      if (lane == 0) {
+      if ((be & 31) == lane) {
+        taken |= 1u << (be >> 5);
+        float own = 0.f;
+#pragma unroll
+        for (int i = 0; i < kPerLane; ++i)
+          if (i == (be >> 5)) own = sc[i];
         sel[k] = be;
-        selv[k] = bv;
+        selv[k] = own;       // the unbiased score
       }
     }
     __syncwarp();
 
-    // ---- weights: p = exp(l - m) / s, renormalised over the kept experts
+    // ---- weights: renormalised scores, then the optional dynamic threshold
     float psum = 0.f;
-    for (int k = 0; k < K; ++k) psum += expf(selv[k] - m) / s;
+    for (int k = 0; k < K; ++k) psum += selv[k];
+    float ksum = 0.f;
+    if (a.dyn_threshold > 0.f)
+      for (int k = 0; k < K; ++k) {
+        const float sh = selv[k] / psum;
+        if (k == 0 || sh >= a.dyn_threshold) ksum += sh;
+      }
     const float denom = a.norm ? (psum + 1e-9f) : 1.f;
     for (int k = lane; k < K; k += 32) {
       const int e = sel[k];
-      const float p = expf(selv[k] - m) / s;
-      const float w = a.norm ? p / denom : p;
+      const float p = selv[k];
+      float w = a.norm ? p / denom : p;
+      bool keep = true;
+      if (a.dyn_threshold > 0.f) {
+        const float sh = p / psum;
+        keep = k == 0 || sh >= a.dyn_threshold;
+        w = keep ? sh / ksum : 0.f;
+      }
       const size_t o = static_cast<size_t>(t) * K + k;
       if (a.sel64) a.sel64[o] = e;
       if (a.wout) a.wout[o] = w;
-      if (a.idx32) a.idx32[o] = e;
+      if (a.idx32) a.idx32[o] = keep ? e : E;
       if (a.w32) a.w32[o] = w;
-      if (a.blockcounts) atomicAdd(&hist[e], 1);
+      if (a.slot_kept) a.slot_kept[o] = keep ? 1 : 0;
+      if (keep && a.blockcounts) atomicAdd(&hist[e], 1);
+      if (a.bal_partial) {
+        bal[E + e] += w;
+        bal[2 * E + e] += w > 0.f ? 1.f : 0.f;
+      }
     }
     __syncwarp();
   }
 
-  if (a.blockcounts) {
+  if (a.blockcounts || a.bal_partial) {
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-      a.blockcounts[static_cast<size_t>(blockIdx.x) * E + e] = hist[e];
+    if (a.blockcounts)
+      for (int e = threadIdx.x; e < E; e += blockDim.x)
+        a.blockcounts[static_cast<size_t>(blockIdx.x) * E + e] = hist[e];
+    if (a.bal_partial)
+      for (int i = threadIdx.x; i < 3 * E; i += blockDim.x) {
+        float acc = 0.f;
+        for (int w = 0; w < kWarps; ++w) acc += bal_all[w * 3 * E + i];   // fixed warp order
+        a.bal_partial[static_cast<size_t>(blockIdx.x) * 3 * E + i] = acc;
+      }
   }
 }
 
 template <typename Tin, bool kVec>
 cudaError_t launch_typed(const RouteArgs& a, cudaStream_t s) {
   const int blocks = (a.T + kRouterTokensPerCta - 1) / kRouterTokensPerCta;
-  const size_t smem = sizeof(float) * (a.E + kWarps * a.E) + sizeof(int) * kWarps * a.K +
-                      sizeof(float) * kWarps * a.K;
+  size_t smem = sizeof(float) * (a.E + kWarps * a.E) + sizeof(int) * kWarps * a.K +
+                sizeof(float) * kWarps * a.K;
+  if (a.bal_partial) smem += sizeof(float) * kWarps * 3 * a.E;
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64 || !done[dev]) {
+      err = cudaFuncSetAttribute(router_topk_kernel<Tin, kVec>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+      if (err != cudaSuccess) return err;
+      if (dev >= 0 && dev < 64) done[dev] = true;
+    }
+  }
   router_topk_kernel<Tin, kVec><<<blocks, kWarps * 32, smem, s>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+int router_simt_parts(int T) { return (T + kRouterTokensPerCta - 1) / kRouterTokensPerCta; }
 
 cudaError_t launch_router(const RouteArgs& a, cudaStream_t s) {
   if (a.dt == kBF16) {

@@ -63,6 +63,11 @@ struct Params {
   float* w32;
   int* blockcounts;   // (ceil(T/32), E) or null
   unsigned int* err;
+  int score;               // 0 softmax, 1 sigmoid
+  const float* sel_bias;   // (E) or null
+  float dyn_threshold;     // > 0: on
+  uint8_t* slot_kept;      // (T, K) or null
+  float* bal_partial;      // (m_tiles, 3, E) or null
 };
 
 template <int NPAD>
@@ -227,8 +232,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       m = fmaxf(m, v);
     }
     float s = 0.f;
-    for (int e = 0; e < E; ++e) s += expf(lrow[e] - m);
-    // K rounds of selection
+    if (p.score == 0)
+      for (int e = 0; e < E; ++e) s += expf(lrow[e] - m);
+    // score of expert e: softmax probability or sigmoid of the logit
+    auto score = [&](int e) {
+      const float l = lrow[e];
+      return p.score == 0 ? expf(l - m) / s : 1.f / (1.f + expf(-l));
+    };
+    // ranking key: the logit (monotone in either score) unless a selection
+    // bias is added to the score
+    auto key = [&](int e) { return p.sel_bias ? score(e) + __ldg(p.sel_bias + e) : lrow[e]; };
+    // K rounds of selection; the chosen index goes to sel64 / idx32 and the
+    // unbiased score to the weight buffer until the weights are final
     float* tmpw = p.w32 ? p.w32 : p.wout;
     float lv = INFINITY;
     int le = -1;
@@ -237,7 +252,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       float bv = -INFINITY;
       int be = 0x7fffffff;
       for (int e = 0; e < E; ++e) {
-        const float v = lrow[e];
+        const float v = key(e);
         if (ranks_before(lv, le, v, e) && ranks_before(v, e, bv, be)) {
           bv = v;
           be = e;
@@ -245,14 +260,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       lv = bv;
       le = be;
-      const float pk = expf(bv - m) / s;
+      const float pk = score(be);
       psum += pk;
       if (valid) {
         const size_t o = static_cast<size_t>(t) * p.K + k;
         tmpw[o] = pk;
         if (p.sel64) p.sel64[o] = be;
         if (p.idx32) p.idx32[o] = be;
-        if (p.blockcounts) atomicAdd(&hist[be], 1);
+      }
+    }
+    // weights: renormalised scores, then the optional dynamic threshold
+    // (the leader stays; the kept shares are renormalised to sum to one)
+    float ksum = 0.f;
+    if (valid && p.dyn_threshold > 0.f) {
+      for (int k = 0; k < p.K; ++k) {
+        const float sh = tmpw[static_cast<size_t>(t) * p.K + k] / psum;
+        if (k == 0 || sh >= p.dyn_threshold) ksum += sh;
       }
     }
     if (valid) {
@@ -260,9 +283,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int k = 0; k < p.K; ++k) {
         const size_t o = static_cast<size_t>(t) * p.K + k;
         const float pk = tmpw[o];
-        const float w = p.norm ? pk / denom : pk;
+        const int e = p.idx32 ? p.idx32[o] : static_cast<int>(p.sel64[o]);
+        float w = p.norm ? pk / denom : pk;
+        bool keep = true;
+        if (p.dyn_threshold > 0.f) {
+          const float sh = pk / psum;
+          keep = k == 0 || sh >= p.dyn_threshold;
+          w = keep ? sh / ksum : 0.f;
+        }
         if (p.wout) p.wout[o] = w;
         if (p.w32) p.w32[o] = w;
+        if (p.slot_kept) p.slot_kept[o] = keep ? 1 : 0;
+        if (!keep && p.idx32) p.idx32[o] = E;           // dropped: no row
+        if (keep && p.blockcounts) atomicAdd(&hist[e], 1);
       }
     }
     if (p.blockcounts) {
@@ -270,6 +303,40 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int b = (m0 + wq * 32) / 32;
       if (m0 + wq * 32 < p.T)
         for (int e = lane; e < E; e += 32) p.blockcounts[static_cast<size_t>(b) * E + e] = hist[e];
+    }
+    if (p.bal_partial) {
+      // per-tile column sums of the scores, the gate and gate > 0, each in
+      // row order (deterministic); the 128 epilogue threads share barrier 1
+      const int tid = row;
+      float* bp = p.bal_partial + static_cast<size_t>(blockIdx.x / p.S) * 3 * E;
+      // the row's scores replace its logits (score(e) reads only lrow[e])
+      for (int e = 0; e < E; ++e) lrow[e] = valid ? score(e) : 0.f;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      for (int e = tid; e < E; e += BM) {
+        float acc = 0.f;
+        for (int r = 0; r < BM; ++r) acc += part[r * C::PART_STRIDE + e];
+        bp[e] = acc;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      for (int e = 0; e < E; ++e) lrow[e] = 0.f;
+      if (valid)
+        for (int k = 0; k < p.K; ++k) {
+          const size_t o = static_cast<size_t>(t) * p.K + k;
+          const int e = p.idx32 ? p.idx32[o] : static_cast<int>(p.sel64[o]);
+          const float w = p.w32 ? p.w32[o] : p.wout[o];
+          if (e < E) lrow[e] = w;
+        }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      for (int e = tid; e < E; e += BM) {
+        float g = 0.f, c = 0.f;
+        for (int r = 0; r < BM; ++r) {
+          const float v = part[r * C::PART_STRIDE + e];
+          g += v;
+          c += v > 0.f ? 1.f : 0.f;
+        }
+        bp[E + e] = g;
+        bp[2 * E + e] = c;
+      }
     }
   }
   __syncwarp();
@@ -349,6 +416,11 @@ cudaError_t launch_npad(const RouteArgs& a, cudaStream_t s) {
   p.w32 = a.w32;
   p.blockcounts = a.blockcounts;
   p.err = a.err;
+  p.score = a.score;
+  p.sel_bias = a.sel_bias;
+  p.dyn_threshold = a.dyn_threshold;
+  p.slot_kept = a.slot_kept;
+  p.bal_partial = a.bal_partial;
   const int m_tiles = (a.T + BM - 1) / BM;
   // split D over a cluster when the row tiles alone would leave SMs idle
   int S = 1;
@@ -370,6 +442,8 @@ cudaError_t launch_npad(const RouteArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+int router_tc_parts(int T) { return (T + BM - 1) / BM; }
 
 cudaError_t launch_router_tc(const RouteArgs& a, cudaStream_t s) {
   if (a.E <= 16) return launch_npad<16>(a, s);

@@ -45,8 +45,20 @@ BF16 = 1
 F64 = 2
 NUM_STAGES = 5
 
+SCORE_SOFTMAX = 0
+SCORE_SIGMOID = 1
+SCORE_NAMES = {"softmax": SCORE_SOFTMAX, "sigmoid": SCORE_SIGMOID}
+
 _lock = threading.Lock()
 _lib = None
+
+
+class RouteOpts(ctypes.Structure):
+    """moe_route_opts_t (include/moe.h)."""
+    _fields_ = [("score", ctypes.c_int), ("selection_bias", ctypes.c_void_p),
+                ("dynamic_threshold", ctypes.c_float), ("capacity_factor", ctypes.c_float),
+                ("seq_len", ctypes.c_int64), ("slot_kept", ctypes.c_void_p),
+                ("balance", ctypes.c_void_p)]
 
 
 class MoEError(RuntimeError):
@@ -74,6 +86,13 @@ def lib() -> ctypes.CDLL:
         L.moe_ffn_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, i64,
                                               i64, i64, i32, vp, vp, vp, vp, vp]
         L.moe_ffn_forward_noalloc.restype = i32
+        L.moe_ffn_forward_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, i64, i64,
+                                         i64, i32, vp, vp, vp, vp, vp, sz,
+                                         ctypes.POINTER(RouteOpts), vp]
+        L.moe_ffn_forward_ex.restype = i32
+        L.moe_route_ex.argtypes = [vp, vp, vp, i64, i64, i32, i32, i32, i32, vp, vp, vp,
+                                   ctypes.POINTER(RouteOpts), vp]
+        L.moe_route_ex.restype = i32
         L.moe_route.argtypes = [vp, vp, vp, i64, i64, i32, i32, i32, i32, vp, vp, vp, vp]
         L.moe_route.restype = i32
         L.moe_status_string.argtypes = [i32]
@@ -243,6 +262,77 @@ def ffn_forward_noalloc(x, router, gate_up_proj, down_proj, E: int, K: int, norm
 def noalloc_scratch_bytes() -> int:
     """Size of the static scratch behind ffn_forward_noalloc (32 MiB)."""
     return 32 << 20
+
+
+def _opts(score="softmax", selection_bias=None, dynamic_threshold=0.0, capacity_factor=0.0,
+          seq_len=0, slot_kept=None, balance=None) -> RouteOpts:
+    sc = SCORE_NAMES.get(score, score) if isinstance(score, str) else int(score)
+    if isinstance(sc, str):
+        sc = 99
+    return RouteOpts(int(sc), _ptr(selection_bias), float(dynamic_threshold),
+                     float(capacity_factor), int(seq_len), _ptr(slot_kept), _ptr(balance))
+
+
+def ffn_forward_ex(x, router, gate_up_proj, down_proj, E: int, K: int, norm_topk_prob: bool, act,
+                   out, selected_experts=None, routing_weights=None, router_bias=None, b1=None,
+                   b2=None, router_logits=None, workspace=None, stream=None, **opts) -> None:
+    """moe_ffn_forward_ex: the forward with routing options (score,
+    selection_bias, dynamic_threshold, capacity_factor, seq_len, slot_kept,
+    balance - see include/moe.h)."""
+    import torch
+    D = int(x.shape[-1])
+    T = int(x.numel() // D) if D else 0
+    F = int(down_proj.shape[-1])
+    dt = _dtype_code(x)
+    a = _act_code(act)
+    if dt in (F32, BF16) and a in (ACT_SILU_GATED, ACT_RELU) and 1 <= K <= E and T > 0:
+        wdt = x.dtype
+        gu_rows = 2 * F if a == ACT_SILU_GATED else F
+        _expect(router, (E, D), "router", wdt)
+        _expect(gate_up_proj, (E, gu_rows, D), "gate_up_proj", wdt)
+        _expect(down_proj, (E, D, F), "down_proj", wdt)
+        _expect(out, tuple(x.shape), "out", wdt)
+        _expect(selected_experts, (T, K), "selected_experts", torch.int64, False)
+        _expect(routing_weights, (T, K), "routing_weights", torch.float32, False)
+        _expect(router_bias, (E,), "router_bias", torch.float32, False)
+        _expect(b1, (E, F), "b1", torch.float32, False)
+        _expect(b2, (E, D), "b2", torch.float32, False)
+        _expect(router_logits, (T, E), "router_logits", torch.float32, False)
+        _expect(opts.get("selection_bias"), (E,), "selection_bias", torch.float32, False)
+        _expect(opts.get("slot_kept"), (T, K), "slot_kept", torch.uint8, False)
+        _expect(opts.get("balance"), (4,), "balance", torch.float32, False)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    o = _opts(**opts)
+    st = lib().moe_ffn_forward_ex(
+        _ptr(x), _ptr(router), _ptr(gate_up_proj), _ptr(down_proj), E, K, int(bool(norm_topk_prob)),
+        a, _ptr(out), _ptr(selected_experts), _ptr(routing_weights), T, D, F, dt,
+        _ptr(router_bias), _ptr(b1), _ptr(b2), _ptr(router_logits), _ptr(workspace), ws_bytes,
+        ctypes.byref(o), _stream(stream))
+    _check(st)
+
+
+def route_ex(x, router, K: int, norm_topk_prob: bool, selected_experts, routing_weights,
+             router_bias=None, router_logits=None, stream=None, **opts) -> None:
+    """moe_route_ex: the router with options (not capacity or balance)."""
+    import torch
+    D = int(x.shape[-1])
+    T = int(x.numel() // D) if D else 0
+    E = int(router.shape[0])
+    dt = _dtype_code(x)
+    if dt in (F32, BF16) and 1 <= K <= E and T > 0:
+        _expect(router, (E, D), "router", x.dtype)
+        _expect(selected_experts, (T, K), "selected_experts", torch.int64)
+        _expect(routing_weights, (T, K), "routing_weights", torch.float32)
+        _expect(router_bias, (E,), "router_bias", torch.float32, False)
+        _expect(router_logits, (T, E), "router_logits", torch.float32, False)
+        _expect(opts.get("selection_bias"), (E,), "selection_bias", torch.float32, False)
+        _expect(opts.get("slot_kept"), (T, K), "slot_kept", torch.uint8, False)
+    o = _opts(**opts)
+    st = lib().moe_route_ex(_ptr(x), _ptr(router), _ptr(router_bias), T, D, E, K,
+                            int(bool(norm_topk_prob)), dt, _ptr(router_logits),
+                            _ptr(selected_experts), _ptr(routing_weights), ctypes.byref(o),
+                            _stream(stream))
+    _check(st)
 
 
 def route(x, router, K: int, norm_topk_prob: bool, selected_experts, routing_weights,

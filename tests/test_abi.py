@@ -118,3 +118,38 @@ def test_workspace_size(L):
     big = moe.workspace_size(4096, 4096, 14336, 8, 2, moe.BF16)
     assert big >= 8192 * (4096 + 14336 + 4096) * 2
     assert big < 8192 * (4096 + 14336 + 4096) * 2 + 8 * 1024 * 1024
+
+
+def test_route_opts_layout_matches_the_header(tmp_path):
+    """The ctypes mirror of moe_route_opts_t has the C layout (gcc)."""
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "moe.h"\n'
+                   'int main(void){printf("%zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(moe_route_opts_t),'
+                   'offsetof(moe_route_opts_t, score), offsetof(moe_route_opts_t, selection_bias),'
+                   'offsetof(moe_route_opts_t, dynamic_threshold), offsetof(moe_route_opts_t, capacity_factor),'
+                   'offsetof(moe_route_opts_t, seq_len), offsetof(moe_route_opts_t, slot_kept),'
+                   'offsetof(moe_route_opts_t, balance)); return 0;}\n')
+    exe = tmp_path / "layout"
+    import subprocess
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
+    R = moe.RouteOpts
+    want = [ctypes.sizeof(R), R.score.offset, R.selection_bias.offset, R.dynamic_threshold.offset,
+            R.capacity_factor.offset, R.seq_len.offset, R.slot_kept.offset, R.balance.offset]
+    assert got == want
+
+
+def test_route_opts_rejected_on_host(L):
+    def fwd(**o):
+        opts = moe._opts(**o)
+        return L.moe_ffn_forward_ex(P, P, P, P, 8, 2, 1, 0, P, P, P, 64, 64, 128, 0, None, None,
+                                    None, None, P, 1 << 40, ctypes.byref(opts), None)
+    assert fwd(score=5) == moe.MOE_ERR_INVALID_ARG
+    assert fwd(dynamic_threshold=-0.1) == moe.MOE_ERR_INVALID_ARG
+    assert fwd(dynamic_threshold=float("nan")) == moe.MOE_ERR_INVALID_ARG
+    assert fwd(capacity_factor=-1.0) == moe.MOE_ERR_INVALID_ARG
+    assert fwd(capacity_factor=1.0, seq_len=48) == moe.MOE_ERR_INVALID_ARG   # not a multiple of 32
+    assert fwd(selection_bias=MIS) == moe.MOE_ERR_ALIGNMENT
+    opts = moe._opts(capacity_factor=1.0)
+    assert L.moe_route_ex(P, P, None, 64, 64, 8, 2, 1, 0, None, P, P, ctypes.byref(opts),
+                          None) == moe.MOE_ERR_INVALID_ARG
