@@ -273,9 +273,27 @@ def run_ours(args, w):
     wts = torch.empty(w.T, w.K, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    ext = dict(score=args.score, dynamic_threshold=args.dynamic_threshold,
+               capacity_factor=args.capacity_factor, seq_len=args.seq_len)
+    if args.selection_bias > 0:
+        sb = np.random.default_rng(7).normal(0, args.selection_bias, w.E).astype(np.float32)
+        ext["selection_bias"] = torch.from_numpy(sb).to(dev)
+    kept = torch.empty(w.T, w.K, dtype=torch.uint8, device=dev)
+    bal = torch.empty(4, dtype=torch.float32, device=dev)
+    use_ext = (args.score != "softmax" or args.selection_bias > 0 or args.dynamic_threshold > 0
+               or args.capacity_factor > 0 or args.balance)
+    if use_ext:
+        ext["slot_kept"] = kept
+        if args.balance:
+            ext["balance"] = bal
+
     def step(xin=x, o=out):
-        moe.ffn_forward(xin, router, gu, dn, w.E, w.K, w.norm_topk_prob, act, o, sel, wts, rb, b1,
-                        b2, None, ws, stream)
+        if use_ext:
+            moe.ffn_forward_ex(xin, router, gu, dn, w.E, w.K, w.norm_topk_prob, act, o, sel, wts,
+                               rb, b1, b2, None, ws, stream, **ext)
+        else:
+            moe.ffn_forward(xin, router, gu, dn, w.E, w.K, w.norm_topk_prob, act, o, sel, wts, rb,
+                            b1, b2, None, ws, stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -284,6 +302,13 @@ def run_ours(args, w):
         raise RuntimeError(f"device status after warm-up: {moe.status_string(st)}")
     load = np.bincount(sel.cpu().numpy().ravel(), minlength=w.E)
     touched = int((load > 0).sum())
+    ext_stats = {}
+    if use_ext:
+        k = kept.cpu().numpy()
+        ext_stats["slots_kept_frac"] = round(float(k.mean()), 4)
+        if args.balance:
+            ext_stats["balance"] = dict(zip(("switch", "gshard", "master", "gshard_probs"),
+                                            [round(float(v), 6) for v in bal.cpu().numpy()]))
 
     # ---------------- timed region: K forwards, device events on the stream
     if world > 1:
@@ -371,7 +396,12 @@ def run_ours(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded, shapes of the pages' workloads; random-init weights)",
-        "config": dict(workload_config(w, world), gemm=args.gemm),
+        "config": dict(workload_config(w, world), gemm=args.gemm,
+                       **({"routing": {"score": args.score, "selection_bias_std": args.selection_bias,
+                                       "dynamic_threshold": args.dynamic_threshold,
+                                       "capacity_factor": args.capacity_factor,
+                                       "seq_len": args.seq_len, "balance": args.balance}}
+                          if use_ext else {})),
         "routed_tflops": round(world * rflops / (ms_step / 1e3) / 1e12, 2),
         "frac_of_bf16_peak": {
             "measured_burst": round(rflops / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
@@ -383,7 +413,7 @@ def run_ours(args, w):
                 "frac_of_nominal_8tbs": round(abytes / (ms_step / 1e3) / 1e9 / NOMINAL["hbm_gbs"], 4)},
         "stages_ms": {k: round(v, 4) for k, v in per_call.items()},
         "dominant_stage": dom,
-        "expert_load": load.tolist(), "experts_touched": touched,
+        "expert_load": load.tolist(), "experts_touched": touched, **ext_stats,
         "roofline": roof,
         "e2e": {"value": round(e_tokens_per_s, 1), "unit": UNIT,
                 "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
@@ -467,6 +497,13 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm", choices=["auto", "1sm", "2sm"], default="auto",
                     help="bf16 grouped GEMM: automatic, one CTA per tile, or CTA pairs")
+    ap.add_argument("--score", choices=["softmax", "sigmoid"], default="softmax")
+    ap.add_argument("--selection-bias", type=float, default=0.0,
+                    help="std of a seeded per-expert selection-only bias (0: none)")
+    ap.add_argument("--dynamic-threshold", type=float, default=0.0)
+    ap.add_argument("--capacity-factor", type=float, default=0.0)
+    ap.add_argument("--seq-len", type=int, default=0)
+    ap.add_argument("--balance", action="store_true", help="also compute the balancing statistics")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     w = synth.WORKLOADS[args.workload]

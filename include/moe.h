@@ -261,6 +261,17 @@ MOE_API moe_status_t moe_ffn_forward_noalloc(const void* x, const void* router,
 #define MOE_GEMM_2SM 2
 MOE_API int moe_set_gemm_mode(int mode);
 
+/*
+ * Whether the bf16 gate_up GEMM fetches its token rows from x by index
+ * (TMA tile::gather4, four rows per copy) instead of from an expert-sorted
+ * copy written by a separate gather kernel.  Results are bit-identical.
+ * Off by default: on B200 the four-row copies deliver the A operand far
+ * slower than the tensor cores consume it (gate_up about 3x slower on the
+ * Mixtral-shaped layer); it saves the gather kernel and its HBM write.
+ * Returns the previous setting.
+ */
+MOE_API int moe_set_fused_gather(int on);
+
 /* Short English description of a status code (static storage). */
 MOE_API const char* moe_status_string(moe_status_t status);
 
@@ -276,6 +287,16 @@ MOE_API int moe_abi_version(void);
  * Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_CUDA.
  */
 MOE_API moe_status_t moe_device_status(void* stream);
+
+/*
+ * Test hook for failure detection: launches one CTA that waits, through the
+ * same bounded mbarrier wait the kernels use, on a barrier nothing ever
+ * arrives at.  The wait gives up after timeout_ms, sets the device error
+ * word and the kernel returns; moe_device_status then reports
+ * MOE_ERR_TIMEOUT and clears the word, and the context stays usable.
+ * timeout_ms must be in [1, 2000].
+ */
+MOE_API moe_status_t moe_debug_bounded_wait(int timeout_ms, void* stream);
 
 /*
  * Stage profiler.  While enabled, moe_ffn_forward records CUDA events

@@ -55,6 +55,8 @@ constexpr uint32_t TMEM_COLS = 512;
 enum { kSiluGated = 0, kReluBias = 1, kBias = 2 };
 
 struct Params {
+  const int* perm;      // gathered A: sorted row -> (token, slot); null otherwise
+  int K;                // slots per token (gathered A)
   const int* offsets;   // (E + 1) first sorted row of each expert
   int E;
   int n_out;            // output columns
@@ -123,7 +125,20 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* rowp, int col0, int n
   }
 }
 
-template <int EPI>
+// Four rows of x (token indices r0..r3), 64 columns from c0, into 512
+// contiguous bytes of shared memory with the same 128-byte swizzle as a
+// tiled load (the tensor map's box is 64 x 1).
+__device__ __forceinline__ void tma_gather4(const CUtensorMap* map, uint64_t* bar, void* dst, int c0,
+                                            int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
+      "r"(r3)
+      : "memory");
+}
+
+template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB, const Params p) {
@@ -182,39 +197,59 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t used = 0, last_parity = 0;   // per stage: ever filled / parity of last fill
-      for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-        int e, m_blk, n_blk;
-        decode_tile(st, E, t, e, m_blk, n_blk);
-        const int rowA = st->off[e] + m_blk * BM;
-        int rowB0, rowB1;
-        if (EPI == kSiluGated) {
-          rowB0 = e * p.b_rows + n_blk * 128;
-          rowB1 = rowB0 + p.up_off;
-        } else {
-          rowB0 = e * p.b_rows + n_blk * 256;
-          rowB1 = rowB0 + 128;
+    // Lane 0 waits for free stages and posts the expected bytes; with a
+    // gathered A every lane then fetches 4 of the tile's 128 token rows.
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t used = 0, last_parity = 0;   // per stage: ever filled / parity of last fill
+    const int rows_live = st->off[E];
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      if (!__shfl_sync(0xffffffffu, lane == 0 ? static_cast<int>(!*abort) : 0, 0)) break;
+      int e, m_blk, n_blk;
+      decode_tile(st, E, t, e, m_blk, n_blk);
+      const int rowA = st->off[e] + m_blk * BM;
+      int rowB0, rowB1;
+      if (EPI == kSiluGated) {
+        rowB0 = e * p.b_rows + n_blk * 128;
+        rowB1 = rowB0 + p.up_off;
+      } else {
+        rowB0 = e * p.b_rows + n_blk * 256;
+        rowB1 = rowB0 + 128;
+      }
+      int tok[4] = {0, 0, 0, 0};
+      if (GATHER) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = rowA + 4 * lane + i;
+          tok[i] = r < rows_live ? __ldg(p.perm + r) / p.K : 0;   // rows past the end: any row
         }
-        bool ok = true;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err)) { ok = false; break; }
-          mbar_arrive_expect_tx(&st->full[stage], STAGE_BYTES);
-          tma_load_2d(&tmA, &st->full[stage], sA + stage * A_BYTES, kb * BK, rowA);
+      }
+      bool ok = true;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        int good = 1;
+        if (lane == 0) {
+          good = mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err) ? 1 : 0;
+          if (good) mbar_arrive_expect_tx(&st->full[stage], STAGE_BYTES);
+        }
+        if (!__shfl_sync(0xffffffffu, good, 0)) { ok = false; break; }
+        if (GATHER)
+          tma_gather4(&tmA, &st->full[stage], sA + stage * A_BYTES + lane * 512, kb * BK, tok[0],
+                      tok[1], tok[2], tok[3]);
+        if (lane == 0) {
+          if (!GATHER) tma_load_2d(&tmA, &st->full[stage], sA + stage * A_BYTES, kb * BK, rowA);
           tma_load_2d(&tmB, &st->full[stage], sB + stage * B_BYTES, kb * BK, rowB0);
           tma_load_2d(&tmB, &st->full[stage], sB + stage * B_BYTES + B_BYTES / 2, kb * BK, rowB1);
           used |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
-      // let every issued load land before the CTA can leave
+      if (!ok) break;
+    }
+    // let every issued load land before the CTA can leave
+    if (lane == 0)
       for (int s = 0; s < STAGES; ++s)
         if (used & (1u << s)) drain_wait(&st->full[s], (last_parity >> s) & 1u, p.err);
-    }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
@@ -347,19 +382,20 @@ EncodeTiledFn encode_fn() {
 
 // Row-major (rows, cols) bf16 matrix, boxes of 128 rows x 64 columns with
 // the 128-byte swizzle; out-of-range elements read as zero.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+              uint32_t box_rows = 128u) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), 128u};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
   const cuuint32_t estr[2] = {1u, 1u};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI>
+template <int EPI, bool GATHER>
 cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params& p, int grid,
                        cudaStream_t s) {
   // the shared-memory opt-in is a per-device function attribute
@@ -371,14 +407,14 @@ cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params&
   {
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= 64 || !done[dev]) {
-      err = cudaFuncSetAttribute(grouped_gemm_tc_kernel<EPI>,
+      err = cudaFuncSetAttribute(grouped_gemm_tc_kernel<EPI, GATHER>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kSmemBytes));
       if (err != cudaSuccess) return err;
       if (dev >= 0 && dev < 64) done[dev] = true;
     }
   }
-  grouped_gemm_tc_kernel<EPI><<<grid, THREADS, kSmemBytes, s>>>(a, b, p);
+  grouped_gemm_tc_kernel<EPI, GATHER><<<grid, THREADS, kSmemBytes, s>>>(a, b, p);
   return cudaGetLastError();
 }
 
@@ -386,12 +422,17 @@ cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params&
 
 cudaError_t launch_gemm_tc(int act, const void* A, int a_rows, const void* W, const int* offsets,
                            int E, int T, int Kdim, int N, int w_rows_per_expert, const float* bias,
-                           void* C, unsigned int* err, cudaStream_t s) {
+                           void* C, unsigned int* err, cudaStream_t s, const int* gather_perm,
+                           int gather_K, int gather_rows) {
   CUtensorMap ma, mb;
-  if (!make_map(&ma, A, static_cast<uint64_t>(a_rows), static_cast<uint64_t>(Kdim)) ||
+  const bool gather = gather_perm != nullptr;
+  if (!make_map(&ma, A, static_cast<uint64_t>(gather ? gather_rows : a_rows),
+                static_cast<uint64_t>(Kdim), gather ? 1u : 128u) ||
       !make_map(&mb, W, static_cast<uint64_t>(E) * w_rows_per_expert, static_cast<uint64_t>(Kdim)))
     return cudaErrorInvalidValue;
   Params p;
+  p.perm = gather_perm;
+  p.K = gather_K;
   p.offsets = offsets;
   p.E = E;
   p.n_out = N;
@@ -407,9 +448,14 @@ cudaError_t launch_gemm_tc(int act, const void* A, int a_rows, const void* W, co
   const long long tiles_bound =
       (static_cast<long long>(a_rows) / BM + E) * ((N + bn_out - 1) / bn_out);
   const int grid = static_cast<int>(tiles_bound < num_sms() ? tiles_bound : num_sms());
-  if (act == kSiluGated) return launch_epi<kSiluGated>(ma, mb, p, grid, s);
-  if (act == kReluBias) return launch_epi<kReluBias>(ma, mb, p, grid, s);
-  return launch_epi<kBias>(ma, mb, p, grid, s);
+  if (gather) {
+    if (act == kSiluGated) return launch_epi<kSiluGated, true>(ma, mb, p, grid, s);
+    if (act == kReluBias) return launch_epi<kReluBias, true>(ma, mb, p, grid, s);
+    return cudaErrorInvalidValue;
+  }
+  if (act == kSiluGated) return launch_epi<kSiluGated, false>(ma, mb, p, grid, s);
+  if (act == kReluBias) return launch_epi<kReluBias, false>(ma, mb, p, grid, s);
+  return launch_epi<kBias, false>(ma, mb, p, grid, s);
 }
 
 }  // namespace moe

@@ -50,6 +50,8 @@ constexpr uint32_t TMEM_COLS = 512;
 enum { kSiluGated = 0, kReluBias = 1, kBias = 2 };
 
 struct Params {
+  const int* perm;    // gathered A: sorted row -> (token, slot); null otherwise
+  int K;
   const int* offsets;
   int E;
   int n_out;
@@ -102,6 +104,17 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(c1)
+      : "memory");
+}
+// Gathered variant: 4 token rows of x (box 64 x 1) into 512 bytes of this
+// CTA's shared memory, completing on the leader's barrier.
+__device__ __forceinline__ void tma_gather4_pair(const CUtensorMap* map, uint32_t bar_cluster_addr,
+                                                 void* dst, int c0, int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
+      ".mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(r0), "r"(r1),
+      "r"(r2), "r"(r3)
       : "memory");
 }
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
@@ -168,7 +181,7 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* rowp, int col0, int n
   }
 }
 
-template <int EPI>
+template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB, const Params p) {
@@ -228,34 +241,58 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Lane 0 waits for free stages (and, in the leader, posts the pair's
+    // expected bytes); with a gathered A every lane fetches 4 of this CTA's
+    // 128 token rows.
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
-      int stage = 0;
-      uint32_t phase = 0, used = 0, last_parity = 0;
-      for (int t = cluster_id; t < total && !*abort; t += num_clusters) {
-        int e, m_blk, n_blk;
-        decode_tile(st, E, t, e, m_blk, n_blk);
-        const int rowA = st->off[e] + m_blk * BMP + static_cast<int>(rank) * BMC;
-        const int rowB = (EPI == kSiluGated)
-                             ? e * p.b_rows + n_blk * 128 + (leader ? 0 : p.up_off)
-                             : e * p.b_rows + n_blk * 256 + static_cast<int>(rank) * 128;
-        bool ok = true;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err)) { ok = false; break; }
-          if (leader) mbar_arrive_expect_tx(&st->full[stage], 2 * STAGE_BYTES);
-          const uint32_t fb = map_to_rank(&st->full[stage], 0);
-          tma_load_2d_pair(&tmA, fb, sA + stage * A_BYTES, kb * BK, rowA);
+    }
+    int stage = 0;
+    uint32_t phase = 0, used = 0, last_parity = 0;
+    const int rows_live = st->off[E];
+    for (int t = cluster_id; t < total; t += num_clusters) {
+      if (!__shfl_sync(0xffffffffu, lane == 0 ? static_cast<int>(!*abort) : 0, 0)) break;
+      int e, m_blk, n_blk;
+      decode_tile(st, E, t, e, m_blk, n_blk);
+      const int rowA = st->off[e] + m_blk * BMP + static_cast<int>(rank) * BMC;
+      const int rowB = (EPI == kSiluGated)
+                           ? e * p.b_rows + n_blk * 128 + (leader ? 0 : p.up_off)
+                           : e * p.b_rows + n_blk * 256 + static_cast<int>(rank) * 128;
+      int tok[4] = {0, 0, 0, 0};
+      if (GATHER) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = rowA + 4 * lane + i;
+          tok[i] = r < rows_live ? __ldg(p.perm + r) / p.K : 0;
+        }
+      }
+      bool ok = true;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        int good = 1;
+        if (lane == 0) {
+          good = mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err) ? 1 : 0;
+          if (good && leader) mbar_arrive_expect_tx(&st->full[stage], 2 * STAGE_BYTES);
+        }
+        if (!__shfl_sync(0xffffffffu, good, 0)) { ok = false; break; }
+        const uint32_t fb = map_to_rank(&st->full[stage], 0);
+        if (GATHER)
+          tma_gather4_pair(&tmA, fb, sA + stage * A_BYTES + lane * 512, kb * BK, tok[0], tok[1],
+                           tok[2], tok[3]);
+        if (lane == 0) {
+          if (!GATHER) tma_load_2d_pair(&tmA, fb, sA + stage * A_BYTES, kb * BK, rowA);
           tma_load_2d_pair(&tmB, fb, sB + stage * B_BYTES, kb * BK, rowB);
           used |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
-      // Let issued loads land before the CTA can leave: the leader sees them
-      // on its full barriers; the peer's complete on the leader's, so the
-      // peer waits for the pair's MMAs to have released its stages.
+      if (!ok) break;
+    }
+    // Let issued loads land before the CTA can leave: the leader sees them
+    // on its full barriers; the peer's complete on the leader's, so the
+    // peer waits for the pair's MMAs to have released its stages.
+    if (lane == 0) {
       int dummy = 0;
       for (int s = 0; s < STAGES; ++s)
         if (used & (1u << s)) {
@@ -397,19 +434,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+              uint32_t box_rows = 128u) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), 128u};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
   const cuuint32_t estr[2] = {1u, 1u};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI>
+template <int EPI, bool GATHER>
 cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params& p, int clusters,
                        cudaStream_t s) {
   static std::mutex mu;
@@ -420,7 +458,7 @@ cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params&
   {
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= 64 || !done[dev]) {
-      err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<EPI>,
+      err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<EPI, GATHER>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kSmemBytes));
       if (err != cudaSuccess) return err;
@@ -439,19 +477,24 @@ cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params&
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<EPI>, a, b, p);
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<EPI, GATHER>, a, b, p);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* W,
                                 const int* offsets, int E, int Kdim, int N, int w_rows_per_expert,
-                                const float* bias, void* C, unsigned int* err, cudaStream_t s) {
+                                const float* bias, void* C, unsigned int* err, cudaStream_t s,
+                                const int* gather_perm, int gather_K, int gather_rows) {
   CUtensorMap ma, mb;
-  if (!make_map(&ma, A, static_cast<uint64_t>(a_rows), static_cast<uint64_t>(Kdim)) ||
+  const bool gather = gather_perm != nullptr;
+  if (!make_map(&ma, A, static_cast<uint64_t>(gather ? gather_rows : a_rows),
+                static_cast<uint64_t>(Kdim), gather ? 1u : 128u) ||
       !make_map(&mb, W, static_cast<uint64_t>(E) * w_rows_per_expert, static_cast<uint64_t>(Kdim)))
     return cudaErrorInvalidValue;
   Params p;
+  p.perm = gather_perm;
+  p.K = gather_K;
   p.offsets = offsets;
   p.E = E;
   p.n_out = N;
@@ -466,9 +509,14 @@ cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* 
       (static_cast<long long>(a_rows) / BMP + E) * ((N + bn_out - 1) / bn_out);
   const int max_clusters = num_sms() / 2;
   const int clusters = static_cast<int>(tiles_bound < max_clusters ? tiles_bound : max_clusters);
-  if (act == kSiluGated) return launch_epi<kSiluGated>(ma, mb, p, clusters, s);
-  if (act == kReluBias) return launch_epi<kReluBias>(ma, mb, p, clusters, s);
-  return launch_epi<kBias>(ma, mb, p, clusters, s);
+  if (gather) {
+    if (act == kSiluGated) return launch_epi<kSiluGated, true>(ma, mb, p, clusters, s);
+    if (act == kReluBias) return launch_epi<kReluBias, true>(ma, mb, p, clusters, s);
+    return cudaErrorInvalidValue;
+  }
+  if (act == kSiluGated) return launch_epi<kSiluGated, false>(ma, mb, p, clusters, s);
+  if (act == kReluBias) return launch_epi<kReluBias, false>(ma, mb, p, clusters, s);
+  return launch_epi<kBias, false>(ma, mb, p, clusters, s);
 }
 
 }  // namespace moe

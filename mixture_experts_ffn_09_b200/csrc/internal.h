@@ -87,16 +87,27 @@ cudaError_t launch_gemm_simt_f32(int act, const float* A, const float* W, const 
 
 // bf16 grouped GEMMs on the tcgen05 tensor cores (same three epilogues).
 // A: (a_rows, Kdim) bf16 sorted rows; W: (E * w_rows_per_expert, Kdim) bf16.
+// With gather_perm set, A is x itself (gather_rows = T rows) and each tile's
+// rows are fetched by token index perm[row] / gather_K (TMA tile::gather4),
+// so the expert-sorted copy of x is never written.
 cudaError_t launch_gemm_tc(int act, const void* A, int a_rows, const void* W, const int* offsets,
                            int E, int T, int Kdim, int N, int w_rows_per_expert,
-                           const float* bias, void* C, unsigned int* err, cudaStream_t s);
+                           const float* bias, void* C, unsigned int* err, cudaStream_t s,
+                           const int* gather_perm = nullptr, int gather_K = 0,
+                           int gather_rows = 0);
 
 // Same GEMM on CTA pairs (tcgen05 cta_group::2, 256-row tiles).
 cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* W,
                                 const int* offsets, int E, int Kdim, int N, int w_rows_per_expert,
-                                const float* bias, void* C, unsigned int* err, cudaStream_t s);
+                                const float* bias, void* C, unsigned int* err, cudaStream_t s,
+                                const int* gather_perm = nullptr, int gather_K = 0,
+                                int gather_rows = 0);
 
 int num_sms();
+
+// One CTA waiting (bounded) on an mbarrier nothing arrives at.
+cudaError_t launch_bounded_wait_probe(unsigned long long timeout_ns, unsigned int* err,
+                                      cudaStream_t s);
 
 // Sets the message moe_last_error() returns on this host thread.
 void set_last_error(const char* msg);

@@ -25,19 +25,23 @@ namespace {
 thread_local std::string g_last_error;
 
 std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
+std::atomic<int> g_fused_gather{0};
 
 // The tensor-core GEMM for one launch: CTA pairs pay off when experts have
-// enough rows to fill 256-row tiles.
+// enough rows to fill 256-row tiles.  With gather_perm the A rows are read
+// from x by token index inside the GEMM.
 cudaError_t launch_gemm_bf16(int act, const void* A, int a_rows, const void* W,
                              const int* offsets, int E, int T, int K, int Kdim, int N,
                              int w_rows, const float* bias, void* C, unsigned int* err,
-                             cudaStream_t s) {
+                             cudaStream_t s, const int* gather_perm = nullptr) {
   const int mode = g_gemm_mode.load();
   const bool pair = mode == MOE_GEMM_2SM ||
                     (mode == MOE_GEMM_AUTO && static_cast<long long>(T) * K >= 512LL * E);
   if (pair)
-    return moe::launch_gemm_tc_pair(act, A, a_rows, W, offsets, E, Kdim, N, w_rows, bias, C, err, s);
-  return moe::launch_gemm_tc(act, A, a_rows, W, offsets, E, T, Kdim, N, w_rows, bias, C, err, s);
+    return moe::launch_gemm_tc_pair(act, A, a_rows, W, offsets, E, Kdim, N, w_rows, bias, C, err, s,
+                                    gather_perm, K, T);
+  return moe::launch_gemm_tc(act, A, a_rows, W, offsets, E, T, Kdim, N, w_rows, bias, C, err, s,
+                             gather_perm, K, T);
 }
 
 __device__ unsigned int g_device_error;   // per device: bounded waits that gave up
@@ -238,6 +242,8 @@ extern "C" {
 
 int moe_abi_version(void) { return MOE_ABI_VERSION; }
 
+int moe_set_fused_gather(int on) { return g_fused_gather.exchange(on ? 1 : 0); }
+
 int moe_set_gemm_mode(int mode) {
   if (mode != MOE_GEMM_AUTO && mode != MOE_GEMM_1SM && mode != MOE_GEMM_2SM) return -1;
   return g_gemm_mode.exchange(mode);
@@ -386,6 +392,9 @@ moe_status_t moe_ffn_forward_ex(const void* x, const void* router, const void* g
   const int seq_len = opts ? static_cast<int>(opts->seq_len) : 0;
   float* balance_out = opts ? opts->balance : nullptr;
   uint8_t* slot_kept = opts ? opts->slot_kept : nullptr;
+  // bf16: gate_up reads the token rows of x directly (TMA gather), so the
+  // expert-sorted copy is not materialised
+  const bool fused_gather = dt == MOE_BF16 && g_fused_gather.load() != 0;
   const int Ti = static_cast<int>(T), Di = static_cast<int>(D), Fi = static_cast<int>(F);
   const int gu_act = act == MOE_ACT_SILU_GATED ? 0 : 1;
   const int gu_rows = act == MOE_ACT_SILU_GATED ? 2 * Fi : Fi;
@@ -427,14 +436,15 @@ moe_status_t moe_ffn_forward_ex(const void* x, const void* router, const void* g
     if (r != cudaSuccess) return r;
     r = moe::launch_permute_scatter(idx32, bbase, totals, bcount, Ti, K, E, offsets, perm, pos,
                                     slot_kept, s);
-    if (r != cudaSuccess) return r;
+    if (r != cudaSuccess || fused_gather) return r;
     return moe::launch_gather_rows(perm, offsets, E, Ti * K, K, x, Di * elem, xperm, s);
   });
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   if (dt == MOE_BF16) {
     e = timer.run(2, [&] {
-      return launch_gemm_bf16(gu_act, xperm, L.Rpad, gate_up_proj, offsets, E, Ti, K, Di, Fi,
-                              gu_rows, b1, H, dev->err, s);
+      return launch_gemm_bf16(gu_act, fused_gather ? x : xperm, L.Rpad, gate_up_proj, offsets, E,
+                              Ti, K, Di, Fi, gu_rows, b1, H, dev->err, s,
+                              fused_gather ? perm : nullptr);
     });
     if (e != cudaSuccess) return cuda_fail(e, "gate_up launch");
     e = timer.run(3, [&] {
@@ -461,6 +471,19 @@ moe_status_t moe_ffn_forward_ex(const void* x, const void* router, const void* g
                                s);
   });
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  return MOE_OK;
+}
+
+moe_status_t moe_debug_bounded_wait(int timeout_ms, void* stream) {
+  g_last_error.clear();
+  if (timeout_ms < 1 || timeout_ms > 2000)
+    return fail(MOE_ERR_INVALID_ARG, "timeout_ms=%d outside [1, 2000]", timeout_ms);
+  DevInfo* dev = nullptr;
+  moe_status_t st = device_info(&dev);
+  if (st != MOE_OK) return st;
+  cudaError_t e = moe::launch_bounded_wait_probe(static_cast<unsigned long long>(timeout_ms) * 1000000ull,
+                                                 dev->err, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "bounded wait launch");
   return MOE_OK;
 }
 

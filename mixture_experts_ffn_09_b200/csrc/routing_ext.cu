@@ -94,7 +94,28 @@ __global__ void __launch_bounds__(256) balance_finalize_kernel(const float* __re
   }
 }
 
+// The bounded wait of the GEMM and router kernels, on a barrier that never
+// completes: it must give up, record the timeout and let the kernel return.
+__global__ void bounded_wait_probe_kernel(unsigned long long timeout_ns, unsigned int* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort, err, timeout_ns);
+  __syncthreads();
+}
+
 }  // namespace
+
+cudaError_t launch_bounded_wait_probe(unsigned long long timeout_ns, unsigned int* err,
+                                      cudaStream_t s) {
+  bounded_wait_probe_kernel<<<1, 32, 0, s>>>(timeout_ns, err);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_capacity_clamp(int* blockcounts, int B, int E, int T, int K, int seq_len,
                                   float capacity_factor, cudaStream_t s) {

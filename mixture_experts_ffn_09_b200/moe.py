@@ -107,6 +107,10 @@ def lib() -> ctypes.CDLL:
         L.moe_profile_enable.restype = i32
         L.moe_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), i32]
         L.moe_profile_read.restype = i32
+        L.moe_debug_bounded_wait.argtypes = [i32, vp]
+        L.moe_debug_bounded_wait.restype = i32
+        L.moe_set_fused_gather.argtypes = [i32]
+        L.moe_set_fused_gather.restype = i32
         L.moe_set_gemm_mode.argtypes = [i32]
         L.moe_set_gemm_mode.restype = i32
         L.moe_stage_name.argtypes = [i32]
@@ -367,9 +371,21 @@ def set_gemm_mode(mode: int) -> int:
     return prev
 
 
+def set_fused_gather(on: bool) -> bool:
+    """Selects whether the bf16 gate_up GEMM gathers its rows from x itself
+    (TMA gather4) or reads an expert-sorted copy; returns the previous."""
+    return bool(lib().moe_set_fused_gather(int(bool(on))))
+
+
 def device_status(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device status."""
     return int(lib().moe_device_status(_stream(stream)))
+
+
+def debug_bounded_wait(timeout_ms: int, stream=None) -> None:
+    """Launches the failure-detection probe (a bounded wait that must time
+    out); read the outcome with device_status()."""
+    _check(lib().moe_debug_bounded_wait(int(timeout_ms), _stream(stream)))
 
 
 def profile_enable(on: bool = True) -> None:

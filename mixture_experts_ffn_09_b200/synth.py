@@ -122,6 +122,11 @@ MIXTRAL_E2 = _reg(Workload(
     name="mixtral_shape_t2048_d4096_f14336_e2_k2_bf16", T=2048, D=4096, F=14336, E=2, K=2,
     act=ACT_SILU_GATED, dtype="bf16", norm_topk_prob=True, seed=5, x_dist="normal"))
 
+# The same cut with 1024 routed rows per expert, as in the Mixtral layer.
+MIXTRAL_E2_T1024 = _reg(Workload(
+    name="mixtral_shape_t1024_d4096_f14336_e2_k2_bf16", T=1024, D=4096, F=14336, E=2, K=2,
+    act=ACT_SILU_GATED, dtype="bf16", norm_topk_prob=True, seed=5, x_dist="normal"))
+
 # Decode-like weight streaming: 32 tokens, swept over top_k.
 DECODE = {k: _reg(Workload(
     name=f"decode_t32_d4096_f14336_e8_k{k}_bf16", T=32, D=4096, F=14336, E=8,

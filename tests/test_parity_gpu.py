@@ -272,3 +272,38 @@ def test_binding_rejects_before_launch():
     assert ei.value.status == moe.MOE_ERR_DTYPE
     torch.cuda.synchronize()
     assert (out == 7.0).all()     # nothing was launched
+
+
+def test_bounded_wait_times_out_and_the_context_survives():
+    """Failure detection without a fault: a bounded wait on a barrier that
+    nothing completes gives up after 50 ms, the device error word reports
+    the timeout (and is cleared), and a forward afterwards is correct."""
+    import time
+    from mixture_experts_ffn_09_b200 import moe
+    assert moe.device_status() == moe.MOE_OK
+    t0 = time.perf_counter()
+    moe.debug_bounded_wait(50)
+    assert moe.device_status() == moe.MOE_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 10.0
+    assert moe.device_status() == moe.MOE_OK       # the word was cleared
+    w = synth.SILU_SMALL
+    _full_check(synth.make_inputs(w), w.E, w.K, w.norm_topk_prob, w.act, w.dtype)
+
+
+@pytest.mark.parametrize("gemm_mode", MODES, indirect=True)
+@pytest.mark.parametrize("act", ["silu_gated", "relu"])
+def test_fused_gather_equals_materialised_rows(gemm_mode, act):
+    """gate_up fetching token rows from x by index (TMA gather4) gives the
+    bit-identical result of reading an expert-sorted copy of x."""
+    from mixture_experts_ffn_09_b200 import moe
+    d = synth.random_case(81, 700, 264, 200, 6, act=act, dtype="bf16", weight_std=0.05)
+    dev = PL.to_device(d)
+    prev = moe.set_fused_gather(False)
+    try:
+        a = PL.run_gpu(dev, 6, 3, True, act)
+        moe.set_fused_gather(True)
+        b = PL.run_gpu(dev, 6, 3, True, act)
+    finally:
+        moe.set_fused_gather(prev)
+    for k in ("out", "sel", "w"):
+        np.testing.assert_array_equal(a[k], b[k])
