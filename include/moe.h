@@ -272,6 +272,15 @@ MOE_API int moe_set_gemm_mode(int mode);
  */
 MOE_API int moe_set_fused_gather(int on);
 
+/*
+ * Whether the kernels of one forward are launched with programmatic
+ * dependent launch (on by default): each kernel's set-up (barriers, tensor
+ * memory, descriptor prefetch) overlaps the end of the previous kernel, and
+ * it waits for that kernel before reading or writing shared buffers.  Same
+ * results either way.  Returns the previous setting.
+ */
+MOE_API int moe_set_pdl(int on);
+
 /* Short English description of a status code (static storage). */
 MOE_API const char* moe_status_string(moe_status_t status);
 

@@ -7,7 +7,8 @@
 // is written exactly once, the K terms are summed in fp32 in slot order and
 // rounded once to the output dtype: no atomics, bitwise repeatable.
 //
-// HBM-bound gather: one CTA per token, 16-byte loads and stores.
+// HBM-bound gather: one CTA per (token, 1024-column chunk), 16-byte loads
+// and stores, so small batches still spread over the SMs.
 #include "common.cuh"
 #include "internal.h"
 
@@ -34,13 +35,16 @@ __global__ void __launch_bounds__(kThreads) combine_bf16_kernel(const __nv_bfloa
                                                                 __nv_bfloat16* __restrict__ out) {
   __shared__ int sp[kMaxExperts];
   __shared__ float sw[kMaxExperts];
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x;
   for (int k = threadIdx.x; k < K; k += kThreads) {
     sp[k] = pos[static_cast<size_t>(t) * K + k];
     sw[k] = w[static_cast<size_t>(t) * K + k];
   }
   __syncthreads();
-  for (int d = threadIdx.x * 8; d < D; d += kThreads * 8) {
+  const int d_hi = min(D, static_cast<int>(blockIdx.y + 1) * kThreads * 8);
+  for (int d = blockIdx.y * kThreads * 8 + threadIdx.x * 8; d < d_hi; d += kThreads * 8) {
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -66,13 +70,16 @@ __global__ void __launch_bounds__(kThreads) combine_f32_kernel(const float* __re
                                                                int D, float* __restrict__ out) {
   __shared__ int sp[kMaxExperts];
   __shared__ float sw[kMaxExperts];
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x;
   for (int k = threadIdx.x; k < K; k += kThreads) {
     sp[k] = pos[static_cast<size_t>(t) * K + k];
     sw[k] = w[static_cast<size_t>(t) * K + k];
   }
   __syncthreads();
-  for (int d = threadIdx.x; d < D; d += kThreads) {
+  const int d_hi = min(D, static_cast<int>(blockIdx.y + 1) * kThreads * 8);
+  for (int d = blockIdx.y * kThreads * 8 + threadIdx.x; d < d_hi; d += kThreads) {
     float acc = 0.f;
     for (int k = 0; k < K; ++k)
       if (sp[k] >= 0) acc = fmaf(sw[k], __ldg(Y + static_cast<size_t>(sp[k]) * D + d), acc);
@@ -84,12 +91,14 @@ __global__ void __launch_bounds__(kThreads) combine_f32_kernel(const float* __re
 
 cudaError_t launch_combine(const void* Y, const float* w32, const int* pos, int T, int K, int D,
                            int dt, void* out, cudaStream_t s) {
+  const dim3 grid(T, (D + kThreads * 8 - 1) / (kThreads * 8));
   if (dt == kBF16) {
-    combine_bf16_kernel<<<T, kThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(Y), w32, pos, K,
-                                               D, static_cast<__nv_bfloat16*>(out));
+    return launch_k(combine_bf16_kernel, grid, dim3(kThreads), 0, s, pdl_enabled(), 1,
+                    static_cast<const __nv_bfloat16*>(Y), w32, pos, K, D,
+                    static_cast<__nv_bfloat16*>(out));
   } else {
-    combine_f32_kernel<<<T, kThreads, 0, s>>>(static_cast<const float*>(Y), w32, pos, K, D,
-                                              static_cast<float*>(out));
+    return launch_k(combine_f32_kernel, grid, dim3(kThreads), 0, s, pdl_enabled(), 1,
+                    static_cast<const float*>(Y), w32, pos, K, D, static_cast<float*>(out));
   }
   return cudaGetLastError();
 }

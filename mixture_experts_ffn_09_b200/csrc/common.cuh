@@ -8,7 +8,13 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace moe {
+
+// Programmatic dependent launch between the kernels of a forward (process
+// wide, on by default; see moe_set_pdl).
+bool pdl_enabled();
 
 // Error bits a kernel ORs into the per-device error word.
 enum : unsigned int { DEVERR_TIMEOUT = 1u, DEVERR_BOUNDS = 2u };
@@ -38,6 +44,45 @@ __device__ __forceinline__ unsigned long long globaltimer() {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ------------------------------------------- programmatic dependent launch
+// Every kernel of a forward lets the next one launch as soon as all of its
+// CTAs have started, and waits for the previous one to finish (and its
+// writes to be visible) before it touches global memory another kernel
+// writes.  Both are no-ops for a grid launched without the attribute.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Host: launches `kernel` with programmatic stream serialization when
+// `pdl` is set, and as a cluster of `cluster_x` CTAs when > 1.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t s, bool pdl, int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // ------------------------------------------------------------- mbarrier

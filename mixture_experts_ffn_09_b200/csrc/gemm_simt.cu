@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(256) gemm_simt_f32_kernel(const float* __restr
   __shared__ float As[BT][BT + 1];
   __shared__ float Gs[BT][BT + 1];
   __shared__ float Us[ACT == 0 ? BT : 1][BT + 1];
+  pdl_trigger();
+  pdl_wait();
   const int e = blockIdx.z;
   const int r0 = offsets[e];
   const int cnt = offsets[e + 1] - r0;
@@ -97,11 +99,14 @@ cudaError_t launch_gemm_simt_f32(int act, const float* A, const float* W, const 
                                  float* C, cudaStream_t s) {
   const dim3 grid((T + BT - 1) / BT, (N + BT - 1) / BT, E);
   if (act == 0)
-    gemm_simt_f32_kernel<0><<<grid, 256, 0, s>>>(A, W, offsets, Kdim, N, w_rows_per_expert, bias, C);
+    return launch_k(gemm_simt_f32_kernel<0>, grid, dim3(256), 0, s, pdl_enabled(), 1, A, W, offsets,
+                    Kdim, N, w_rows_per_expert, bias, C);
   else if (act == 1)
-    gemm_simt_f32_kernel<1><<<grid, 256, 0, s>>>(A, W, offsets, Kdim, N, w_rows_per_expert, bias, C);
+    return launch_k(gemm_simt_f32_kernel<1>, grid, dim3(256), 0, s, pdl_enabled(), 1, A, W, offsets,
+                    Kdim, N, w_rows_per_expert, bias, C);
   else
-    gemm_simt_f32_kernel<2><<<grid, 256, 0, s>>>(A, W, offsets, Kdim, N, w_rows_per_expert, bias, C);
+    return launch_k(gemm_simt_f32_kernel<2>, grid, dim3(256), 0, s, pdl_enabled(), 1, A, W, offsets,
+                    Kdim, N, w_rows_per_expert, bias, C);
   return cudaGetLastError();
 }
 

@@ -165,6 +165,20 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(&st->mma_done, 1);
     st->abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&st->tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  pdl_trigger();
+  // the expert offsets come from the permutation kernel
+  pdl_wait();
+  if (threadIdx.x == 0) {
     int acc = 0;
     for (int e = 0; e < E; ++e) {
       const int o0 = p.offsets[e], o1 = p.offsets[e + 1];
@@ -177,15 +191,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     st->off[E] = p.offsets[E];
     st->tile_start[E] = acc;
     st->total_tiles = acc;
-    mbar_fence_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-  }
-  if (warp == 1) {
-    tmem_alloc(&st->tmem_base, TMEM_COLS);
-    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
@@ -414,8 +419,8 @@ cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params&
       if (dev >= 0 && dev < 64) done[dev] = true;
     }
   }
-  grouped_gemm_tc_kernel<EPI, GATHER><<<grid, THREADS, kSmemBytes, s>>>(a, b, p);
-  return cudaGetLastError();
+  return launch_k(grouped_gemm_tc_kernel<EPI, GATHER>, dim3(grid), dim3(THREADS), kSmemBytes, s,
+                  pdl_enabled(), 1, a, b, p);
 }
 
 }  // namespace

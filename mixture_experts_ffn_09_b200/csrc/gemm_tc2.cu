@@ -212,6 +212,20 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(&st->mma_done, 1);
     st->abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&st->tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  pdl_trigger();
+  // the expert offsets come from the permutation kernel
+  pdl_wait();
+  if (threadIdx.x == 0) {
     int acc = 0;
     for (int e = 0; e < E; ++e) {
       const int o0 = p.offsets[e], o1 = p.offsets[e + 1];
@@ -224,11 +238,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     st->off[E] = p.offsets[E];
     st->tile_start[E] = acc;
     st->total_tiles = acc;
-    mbar_fence_init();
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(&st->tmem_base, TMEM_COLS);
-    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
@@ -244,10 +253,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     // Lane 0 waits for free stages (and, in the leader, posts the pair's
     // expected bytes); with a gathered A every lane fetches 4 of this CTA's
     // 128 token rows.
-    if (lane == 0) {
-      tma_prefetch_desc(&tmA);
-      tma_prefetch_desc(&tmB);
-    }
     int stage = 0;
     uint32_t phase = 0, used = 0, last_parity = 0;
     const int rows_live = st->off[E];
@@ -465,19 +470,8 @@ cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params&
       if (dev >= 0 && dev < 64) done[dev] = true;
     }
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * clusters);
-  cfg.blockDim = dim3(THREADS);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<EPI, GATHER>, a, b, p);
+  return launch_k(grouped_gemm_pair_kernel<EPI, GATHER>, dim3(2 * clusters), dim3(THREADS),
+                  kSmemBytes, s, pdl_enabled(), 2, a, b, p);
 }
 
 }  // namespace

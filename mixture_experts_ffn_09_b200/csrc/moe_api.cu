@@ -26,6 +26,7 @@ thread_local std::string g_last_error;
 
 std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
 std::atomic<int> g_fused_gather{0};
+std::atomic<int> g_pdl{1};
 
 // The tensor-core GEMM for one launch: CTA pairs pay off when experts have
 // enough rows to fill 256-row tiles.  With gather_perm the A rows are read
@@ -243,6 +244,8 @@ extern "C" {
 int moe_abi_version(void) { return MOE_ABI_VERSION; }
 
 int moe_set_fused_gather(int on) { return g_fused_gather.exchange(on ? 1 : 0); }
+
+int moe_set_pdl(int on) { return g_pdl.exchange(on ? 1 : 0); }
 
 int moe_set_gemm_mode(int mode) {
   if (mode != MOE_GEMM_AUTO && mode != MOE_GEMM_1SM && mode != MOE_GEMM_2SM) return -1;
@@ -534,6 +537,8 @@ int moe_profile_read(float* ms, int n_stages) {
 }  // extern "C"
 
 namespace moe {
+bool pdl_enabled() { return g_pdl.load() != 0; }
+
 int num_sms() {
   int dev = 0;
   cudaGetDevice(&dev);

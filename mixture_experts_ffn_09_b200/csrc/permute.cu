@@ -32,6 +32,8 @@ __global__ void __launch_bounds__(kScanThreads) permute_scan_kernel(const int* _
                                                                     int* __restrict__ totals) {
   __shared__ int wsum[kScanThreads / 32];
   __shared__ int carry;
+  pdl_trigger();
+  pdl_wait();
   const int e = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) carry = 0;
@@ -73,6 +75,8 @@ __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
   __shared__ int kept[kMaxExperts];
   __shared__ int run[kMaxExperts];
   __shared__ int wc[kScatterWarps][kMaxExperts];
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
   if (threadIdx.x == 0) {
@@ -147,6 +151,8 @@ __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const int* 
                                                                      const uint8_t* __restrict__ x,
                                                                      int row_bytes,
                                                                      uint8_t* __restrict__ x_perm) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * (kGatherThreads / 32) + warp;
   if (r >= offsets[E]) return;
@@ -167,27 +173,25 @@ __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const int* 
 
 cudaError_t launch_permute_scan(const int* blockcounts, int B, int E, int* blockbase, int* totals,
                                 cudaStream_t s) {
-  permute_scan_kernel<<<E, kScanThreads, 0, s>>>(blockcounts, B, E, blockbase, totals);
-  return cudaGetLastError();
+  return launch_k(permute_scan_kernel, dim3(E), dim3(kScanThreads), 0, s, pdl_enabled(), 1,
+                  blockcounts, B, E, blockbase, totals);
 }
 
 cudaError_t launch_permute_scatter(const int* idx32, const int* blockbase, const int* totals,
                                    const int* blockcounts, int T, int K, int E, int* offsets,
                                    int* perm, int* pos, uint8_t* slot_kept, cudaStream_t s) {
   const int B = (T + kRouterTokensPerCta - 1) / kRouterTokensPerCta;
-  permute_scatter_kernel<<<B, kScatterThreads, 0, s>>>(idx32, blockbase, totals, blockcounts, T, K,
-                                                        E, offsets, perm, pos, slot_kept);
-  return cudaGetLastError();
+  return launch_k(permute_scatter_kernel, dim3(B), dim3(kScatterThreads), 0, s, pdl_enabled(), 1,
+                  idx32, blockbase, totals, blockcounts, T, K, E, offsets, perm, pos, slot_kept);
 }
 
 cudaError_t launch_gather_rows(const int* perm, const int* offsets, int E, int R_max, int K,
                                const void* x, int row_bytes, void* x_perm, cudaStream_t s) {
   const int rows_per_cta = kGatherThreads / 32;
   const int grid = (R_max + rows_per_cta - 1) / rows_per_cta;
-  gather_rows_kernel<<<grid, kGatherThreads, 0, s>>>(perm, offsets, E, K,
-                                                     static_cast<const uint8_t*>(x), row_bytes,
-                                                     static_cast<uint8_t*>(x_perm));
-  return cudaGetLastError();
+  return launch_k(gather_rows_kernel, dim3(grid), dim3(kGatherThreads), 0, s, pdl_enabled(), 1,
+                  perm, offsets, E, K, static_cast<const uint8_t*>(x), row_bytes,
+                  static_cast<uint8_t*>(x_perm));
 }
 
 }  // namespace moe

@@ -70,6 +70,8 @@ __global__ void __launch_bounds__(kWarps * 32) router_topk_kernel(RouteArgs a) {
   float* bal_all = selv_all + kWarps * K;                      // kWarps * 3 * E (balance only)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_trigger();
+  pdl_wait();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   if (a.bal_partial)
     for (int i = threadIdx.x; i < kWarps * 3 * E; i += blockDim.x) bal_all[i] = 0.f;
@@ -264,8 +266,8 @@ cudaError_t launch_typed(const RouteArgs& a, cudaStream_t s) {
       if (dev >= 0 && dev < 64) done[dev] = true;
     }
   }
-  router_topk_kernel<Tin, kVec><<<blocks, kWarps * 32, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(router_topk_kernel<Tin, kVec>, dim3(blocks), dim3(kWarps * 32), smem, s,
+                  pdl_enabled(), 1, a);
 }
 
 }  // namespace

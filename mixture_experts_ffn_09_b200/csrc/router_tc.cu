@@ -100,12 +100,14 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
 
-// Reads a float at the same shared-memory offset in CTA `rank` of the cluster.
+// Reads a float at the same shared-memory offset in CTA `rank` of the
+// cluster.  No memory clobber: a batch of these issues back to back (the
+// cluster barriers around the reduction order them with the writes).
 __device__ __forceinline__ float ld_dsmem(const float* local, uint32_t rank) {
   uint32_t a = smem_u32(local), r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
   float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(r) : "memory");
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(r));
   return v;
 }
 
@@ -128,6 +130,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int kb_hi = (static_cast<int>(rank) + 1) * p.num_kb / p.S;
   float* part = reinterpret_cast<float*>(sA);   // reuses the ring once the MMAs are done
 
+  pdl_trigger();
   for (int i = threadIdx.x; i < 4 * kMaxExperts; i += THREADS) (&st->hist[0][0])[i] = 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -146,6 +149,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the previous forward's kernels may still read this call's outputs
+  pdl_wait();
   const uint32_t tmem = st->tmem_base;
   volatile int* abort = &st->abort;
 
@@ -220,11 +225,31 @@ __global__ void __launch_bounds__(THREADS, 1)
     const bool valid = t < p.T;
     int* hist = st->hist[wq];
     float* lrow = part + row * C::PART_STRIDE;
-    // sum the split partials in rank order, add the bias, write the logits
+    // sum the split partials in rank order: for 8 experts at a time, all
+    // remote loads are issued before the first add
+    if (p.S > 1) {
+      for (int e0 = 0; e0 < E; e0 += 8) {
+        float rem[7][8];
+#pragma unroll
+        for (int q = 1; q < 8; ++q)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            rem[q - 1][j] = (q < p.S && e0 + j < E) ? ld_dsmem(lrow + e0 + j, q) : 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (e0 + j >= E) break;
+          float v = lrow[e0 + j];
+#pragma unroll
+          for (int q = 1; q < 8; ++q)
+            if (q < p.S) v += rem[q - 1][j];
+          lrow[e0 + j] = v;
+        }
+      }
+    }
+    // add the bias, write the logits
     float m = -INFINITY;
     for (int e = 0; e < E; ++e) {
       float v = lrow[e];
-      for (int q = 1; q < p.S; ++q) v += ld_dsmem(lrow + e, static_cast<uint32_t>(q));
       if (p.bias) v += __ldg(p.bias + e);
       if (valid && p.logits) p.logits[static_cast<size_t>(t) * E + e] = v;
       if (isnan(v)) v = -INFINITY;
@@ -426,19 +451,8 @@ cudaError_t launch_npad(const RouteArgs& a, cudaStream_t s) {
   int S = 1;
   while (S < 8 && m_tiles * S * 2 <= num_sms() && S * 2 <= p.num_kb) S *= 2;
   p.S = S;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(m_tiles * p.S);
-  cfg.blockDim = dim3(THREADS);
-  cfg.dynamicSmemBytes = smem_bytes<NPAD>();
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.S;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = p.S > 1 ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, router_tc_kernel<NPAD>, mx, mw, p);
+  return launch_k(router_tc_kernel<NPAD>, dim3(m_tiles * p.S), dim3(THREADS), smem_bytes<NPAD>(), s,
+                  pdl_enabled(), p.S, mx, mw, p);
 }
 
 }  // namespace

@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(kClampWarps * 32) capacity_clamp_kernel(int* _
                                                                         int B, int E, int T, int K,
                                                                         int blocks_per_seq,
                                                                         float cf) {
+  pdl_trigger();
+  pdl_wait();
   const int seq = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b_lo = seq * blocks_per_seq;
@@ -59,6 +61,8 @@ __global__ void __launch_bounds__(256) balance_finalize_kernel(const float* __re
                                                                int parts, int E, int T,
                                                                float* __restrict__ out) {
   __shared__ float mp[kMaxExperts], mg[kMaxExperts], fr[kMaxExperts];
+  pdl_trigger();
+  pdl_wait();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     float P = 0.f, G = 0.f, C = 0.f;
     for (int i = 0; i < parts; ++i) {
@@ -121,15 +125,14 @@ cudaError_t launch_capacity_clamp(int* blockcounts, int B, int E, int T, int K, 
                                   float capacity_factor, cudaStream_t s) {
   const int bps = seq_len > 0 ? seq_len / kRouterTokensPerCta : B;
   const int seqs = (B + bps - 1) / bps;
-  capacity_clamp_kernel<<<seqs, kClampWarps * 32, 0, s>>>(blockcounts, B, E, T, K, bps,
-                                                          capacity_factor);
-  return cudaGetLastError();
+  return launch_k(capacity_clamp_kernel, dim3(seqs), dim3(kClampWarps * 32), 0, s, pdl_enabled(),
+                  1, blockcounts, B, E, T, K, bps, capacity_factor);
 }
 
 cudaError_t launch_balance_finalize(const float* partial, int parts, int E, int T, float* out4,
                                     cudaStream_t s) {
-  balance_finalize_kernel<<<1, 256, 0, s>>>(partial, parts, E, T, out4);
-  return cudaGetLastError();
+  return launch_k(balance_finalize_kernel, dim3(1), dim3(256), 0, s, pdl_enabled(), 1, partial,
+                  parts, E, T, out4);
 }
 
 }  // namespace moe

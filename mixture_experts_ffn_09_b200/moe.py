@@ -109,6 +109,8 @@ def lib() -> ctypes.CDLL:
         L.moe_profile_read.restype = i32
         L.moe_debug_bounded_wait.argtypes = [i32, vp]
         L.moe_debug_bounded_wait.restype = i32
+        L.moe_set_pdl.argtypes = [i32]
+        L.moe_set_pdl.restype = i32
         L.moe_set_fused_gather.argtypes = [i32]
         L.moe_set_fused_gather.restype = i32
         L.moe_set_gemm_mode.argtypes = [i32]
@@ -369,6 +371,12 @@ def set_gemm_mode(mode: int) -> int:
     if prev < 0:
         raise ValueError(f"unknown GEMM mode {mode}")
     return prev
+
+
+def set_pdl(on: bool) -> bool:
+    """Programmatic dependent launch between a forward's kernels (default
+    on); returns the previous setting."""
+    return bool(lib().moe_set_pdl(int(bool(on))))
 
 
 def set_fused_gather(on: bool) -> bool:
