@@ -196,6 +196,32 @@ def cpu_cores() -> int:
 
 
 # ------------------------------------------------------------------- ranks
+class Watchdog:
+    """Bounded waits for the device work of one rank.
+
+    Every point where the bench waits for the GPU goes through ``sync``: it
+    records an event on the stream and polls it; work that has not finished
+    after ``limit_s`` ends the process with a one-line error naming the phase
+    (process exit tears the context down, so a stalled kernel cannot hold the
+    GPU), instead of blocking until an outside timeout kills the job."""
+
+    def __init__(self, dev, stream, limit_s: float):
+        self.dev, self.stream, self.limit_s = dev, stream, limit_s
+
+    def sync(self, what: str):
+        import torch
+        ev = torch.cuda.Event()
+        ev.record(self.stream)
+        t0 = time.monotonic()
+        while not ev.query():
+            if time.monotonic() - t0 > self.limit_s:
+                print(json.dumps({"error": f"device work of phase '{what}' did not finish within "
+                                           f"{self.limit_s:.0f} s"}), flush=True)
+                os._exit(3)
+            time.sleep(0.0005)
+        torch.cuda.synchronize(self.dev)
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -296,8 +322,10 @@ def run_ours(args, w):
             moe.ffn_forward(xin, router, gu, dn, w.E, w.K, w.norm_topk_prob, act, o, sel, wts, rb,
                             b1, b2, None, ws, stream)
 
-    for _ in range(max(args.warmup, 3)):
+    wd = Watchdog(dev, stream, args.watchdog)
+    for i in range(max(args.warmup, 3)):
         step()
+        wd.sync(f"warm-up step {i}")
     st = moe.device_status(stream)
     if st != moe.MOE_OK:
         raise RuntimeError(f"device status after warm-up: {moe.status_string(st)}")
@@ -315,7 +343,7 @@ def run_ours(args, w):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize(dev)
+    wd.sync("before the timed region")
     clocks = ClockSampler(local)
     clocks.start()
     t0 = torch.cuda.Event(enable_timing=True)
@@ -324,7 +352,7 @@ def run_ours(args, w):
     for _ in range(args.steps):
         step()
     t1.record(stream)
-    torch.cuda.synchronize(dev)
+    wd.sync("timed region")
     clk = clocks.stop()
     local_ms = t0.elapsed_time(t1)
     if world > 1:
@@ -338,7 +366,7 @@ def run_ours(args, w):
     moe.profile_enable(True)
     for _ in range(max(1, min(args.steps, 50))):
         step()
-    torch.cuda.synchronize(dev)
+    wd.sync("per-stage pass")
     stage_ms, calls = moe.profile_read()
     moe.profile_enable(False)
     st = moe.device_status(stream)
@@ -355,7 +383,7 @@ def run_ours(args, w):
         xd.copy_(xh, non_blocking=True)
         step(xd, out)
         oh.copy_(out, non_blocking=True)
-    torch.cuda.synchronize(dev)
+    wd.sync("end-to-end warm-up")
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -364,7 +392,7 @@ def run_ours(args, w):
         step(xd, out)
         oh.copy_(out, non_blocking=True)
     e1.record(stream)
-    torch.cuda.synchronize(dev)
+    wd.sync("end-to-end region")
     e_ms, e_tokens_per_s = throughput(e0.elapsed_time(e1), e_steps, w.T, world, dev)
     io_bytes = w.T * w.D * (2 if dt == moe.BF16 else 4)
 
@@ -514,6 +542,8 @@ def main(argv=None):
     ap.add_argument("--balance", action="store_true", help="also compute the balancing statistics")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch the kernels without programmatic dependent launch")
+    ap.add_argument("--watchdog", type=float, default=120.0,
+                    help="seconds any wait for the device may take before the run is ended")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     w = synth.WORKLOADS[args.workload]

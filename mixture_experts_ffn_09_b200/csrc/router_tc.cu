@@ -18,15 +18,16 @@
 //
 // Streaming x is latency-bound per SM, so few row tiles (small T) would use
 // few SMs: the D axis is then split over a thread-block cluster of S <= 8
-// CTAs.  Each CTA accumulates its share of D in TMEM and copies the partial
-// logits to its shared memory; after a cluster barrier CTA rank 0 adds the S
-// partials in rank order through distributed shared memory (fixed order:
-// deterministic, no atomics, no global workspace) and runs the per-token
-// epilogue.
+// CTAs.  Each CTA accumulates its share of D in TMEM and stores the partial
+// logits into its own slot of rank 0's shared memory (remote stores through
+// distributed shared memory); after a cluster barrier rank 0 adds the S
+// slots in rank order (fixed order: deterministic, no atomics, no global
+// workspace) and runs the per-token epilogue.
 //
-// Top-k without a "taken" set: the k-th choice is the best entry that ranks
+// Top-k: for K <= 8 one pass over the experts keeps a sorted register list
+// of the best K; for larger K, the k-th choice is the best entry that ranks
 // strictly after the (k-1)-th in the order (value descending, index
-// ascending), so each of the K rounds is one scan over the row.
+// ascending), one scan over the row per round.
 #include <math.h>
 
 #include <mutex>
@@ -100,16 +101,16 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
 
-// Reads a float at the same shared-memory offset in CTA `rank` of the
-// cluster.  No memory clobber: a batch of these issues back to back (the
-// cluster barriers around the reduction order them with the writes).
-__device__ __forceinline__ float ld_dsmem(const float* local, uint32_t rank) {
-  uint32_t a = smem_u32(local), r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(r));
-  return v;
+// Address of the same shared-memory offset in cluster rank 0.
+__device__ __forceinline__ uint32_t map_to_rank0(const void* local) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(r) : "r"(smem_u32(local)));
+  return r;
 }
+__device__ __forceinline__ void st_dsmem(uint32_t cluster_addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr), "f"(v) : "memory");
+}
+
 
 template <int NPAD>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -196,55 +197,57 @@ __global__ void __launch_bounds__(THREADS, 1)
       int dummy = 0;
       mbar_wait(&st->mma_done, 0, &dummy, p.err);
     }
-  } else {
-    // -------------------- partial logits: TMEM -> this CTA's shared memory
-    const int wq = warp & 3;
-    const int row = wq * 32 + lane;
-    const uint32_t tb = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    if (mbar_wait(&st->tfull, 0, abort, p.err)) {
+  }
+  // Partial logits of this CTA's k-blocks: the epilogue warps wait for the
+  // MMAs; once every CTA of the cluster is past its MMAs (barrier A, taken
+  // by all threads, so rank 0's ring is free) they store the partials into
+  // slot `rank` of rank 0's shared memory - remote stores for the other
+  // ranks, which do not stall the issuing thread - and barrier B publishes
+  // them to rank 0.
+  const int wq = warp & 3;
+  const int row = wq * 32 + lane;
+  bool have = false;
+  if (warp >= 2) {
+    have = mbar_wait(&st->tfull, 0, abort, p.err);
+    if (have) {
       tc_fence_after();
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      for (int c0 = 0; c0 < E; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tb + c0, r);
-        tmem_ld_wait();
+    }
+  }
+  __syncwarp();
+  if (p.S > 1) cluster_sync_all();                                   // A
+  if (have) {
+    const uint32_t tb = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    float* dst = part + (static_cast<int>(rank) * BM + row) * C::PART_STRIDE;
+    for (int c0 = 0; c0 < E; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tb + c0, r);
+      tmem_ld_wait();
+      if (rank == 0) {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (c0 + j < NPAD) part[row * C::PART_STRIDE + c0 + j] = __uint_as_float(r[j]);
+          if (c0 + j < E) dst[c0 + j] = __uint_as_float(r[j]);
+      } else {
+        const uint32_t d0 = map_to_rank0(dst + c0);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c0 + j < E) st_dsmem(d0 + 4u * j, __uint_as_float(r[j]));
       }
     }
   }
   __syncwarp();
-  if (p.S > 1) cluster_sync_all(); else __syncthreads();
+  if (p.S > 1) cluster_sync_all(); else __syncthreads();            // B
 
   if (warp >= 2 && rank == 0 && !*abort) {
     // ------------------------------------------------ one token per thread
-    const int wq = warp & 3;
-    const int row = wq * 32 + lane;
     const int t = m0 + row;
     const bool valid = t < p.T;
     int* hist = st->hist[wq];
     float* lrow = part + row * C::PART_STRIDE;
-    // sum the split partials in rank order: for 8 experts at a time, all
-    // remote loads are issued before the first add
-    if (p.S > 1) {
-      for (int e0 = 0; e0 < E; e0 += 8) {
-        float rem[7][8];
-#pragma unroll
-        for (int q = 1; q < 8; ++q)
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            rem[q - 1][j] = (q < p.S && e0 + j < E) ? ld_dsmem(lrow + e0 + j, q) : 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (e0 + j >= E) break;
-          float v = lrow[e0 + j];
-#pragma unroll
-          for (int q = 1; q < 8; ++q)
-            if (q < p.S) v += rem[q - 1][j];
-          lrow[e0 + j] = v;
-        }
-      }
+    // sum the split partials in rank order (all local now)
+    for (int q = 1; q < p.S; ++q) {
+      const float* src = part + (q * BM + row) * C::PART_STRIDE;
+      for (int e = 0; e < E; ++e) lrow[e] += src[e];
     }
     // add the bias, write the logits
     float m = -INFINITY;
@@ -267,60 +270,135 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ranking key: the logit (monotone in either score) unless a selection
     // bias is added to the score
     auto key = [&](int e) { return p.sel_bias ? score(e) + __ldg(p.sel_bias + e) : lrow[e]; };
-    // K rounds of selection; the chosen index goes to sel64 / idx32 and the
-    // unbiased score to the weight buffer until the weights are final
-    float* tmpw = p.w32 ? p.w32 : p.wout;
-    float lv = INFINITY;
-    int le = -1;
-    float psum = 0.f;
-    for (int k = 0; k < p.K; ++k) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
+    // K rounds of selection, then the weights.  For K <= 8 the choices stay
+    // in registers; larger K parks them in the output buffers between the
+    // two loops.
+    int se[8];
+    float sw[8];
+    if (p.K <= 8) {
+      // one pass over the experts, bubbling each into a sorted list of the
+      // best K (value descending, index ascending: a later equal value never
+      // overtakes, so the lower index stays ahead)
+      float tv[8];
+      int te[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        tv[k] = -INFINITY;
+        te[k] = 0x7fffffff;
+      }
       for (int e = 0; e < E; ++e) {
-        const float v = key(e);
-        if (ranks_before(lv, le, v, e) && ranks_before(v, e, bv, be)) {
-          bv = v;
-          be = e;
+        float v = key(e);
+        int ve = e;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (k < p.K && ranks_before(v, ve, tv[k], te[k])) {
+            const float sv = tv[k];
+            const int si = te[k];
+            tv[k] = v;
+            te[k] = ve;
+            v = sv;
+            ve = si;
+          }
         }
       }
-      lv = bv;
-      le = be;
-      const float pk = score(be);
-      psum += pk;
-      if (valid) {
-        const size_t o = static_cast<size_t>(t) * p.K + k;
-        tmpw[o] = pk;
-        if (p.sel64) p.sel64[o] = be;
-        if (p.idx32) p.idx32[o] = be;
+      float pk[8];
+      float psum = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (k < p.K) {
+          se[k] = te[k];
+          pk[k] = score(te[k]);
+          psum += pk[k];
+        }
       }
-    }
-    // weights: renormalised scores, then the optional dynamic threshold
-    // (the leader stays; the kept shares are renormalised to sum to one)
-    float ksum = 0.f;
-    if (valid && p.dyn_threshold > 0.f) {
-      for (int k = 0; k < p.K; ++k) {
-        const float sh = tmpw[static_cast<size_t>(t) * p.K + k] / psum;
-        if (k == 0 || sh >= p.dyn_threshold) ksum += sh;
+      float ksum = 0.f;
+      if (p.dyn_threshold > 0.f) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (k < p.K) {
+            const float sh = pk[k] / psum;
+            if (k == 0 || sh >= p.dyn_threshold) ksum += sh;
+          }
       }
-    }
-    if (valid) {
       const float denom = p.norm ? (psum + 1e-9f) : 1.f;
-      for (int k = 0; k < p.K; ++k) {
-        const size_t o = static_cast<size_t>(t) * p.K + k;
-        const float pk = tmpw[o];
-        const int e = p.idx32 ? p.idx32[o] : static_cast<int>(p.sel64[o]);
-        float w = p.norm ? pk / denom : pk;
-        bool keep = true;
-        if (p.dyn_threshold > 0.f) {
-          const float sh = pk / psum;
-          keep = k == 0 || sh >= p.dyn_threshold;
-          w = keep ? sh / ksum : 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (k < p.K) {
+          float w = p.norm ? pk[k] / denom : pk[k];
+          bool keep = true;
+          if (p.dyn_threshold > 0.f) {
+            const float sh = pk[k] / psum;
+            keep = k == 0 || sh >= p.dyn_threshold;
+            w = keep ? sh / ksum : 0.f;
+          }
+          sw[k] = w;
+          if (valid) {
+            const size_t o = static_cast<size_t>(t) * p.K + k;
+            if (p.sel64) p.sel64[o] = se[k];
+            if (p.wout) p.wout[o] = w;
+            if (p.w32) p.w32[o] = w;
+            if (p.idx32) p.idx32[o] = keep ? se[k] : E;   // dropped: no row
+            if (p.slot_kept) p.slot_kept[o] = keep ? 1 : 0;
+            if (keep && p.blockcounts) atomicAdd(&hist[se[k]], 1);
+          }
         }
-        if (p.wout) p.wout[o] = w;
-        if (p.w32) p.w32[o] = w;
-        if (p.slot_kept) p.slot_kept[o] = keep ? 1 : 0;
-        if (!keep && p.idx32) p.idx32[o] = E;           // dropped: no row
-        if (keep && p.blockcounts) atomicAdd(&hist[e], 1);
+      }
+    } else {
+      // the chosen index goes to sel64 / idx32 and the unbiased score to the
+      // weight buffer until the weights are final
+      float* tmpw = p.w32 ? p.w32 : p.wout;
+      float lv = INFINITY;
+      int le = -1;
+      float psum = 0.f;
+      for (int k = 0; k < p.K; ++k) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+        for (int e = 0; e < E; ++e) {
+          const float v = key(e);
+          if (ranks_before(lv, le, v, e) && ranks_before(v, e, bv, be)) {
+            bv = v;
+            be = e;
+          }
+        }
+        lv = bv;
+        le = be;
+        const float pk = score(be);
+        psum += pk;
+        if (valid) {
+          const size_t o = static_cast<size_t>(t) * p.K + k;
+          tmpw[o] = pk;
+          if (p.sel64) p.sel64[o] = be;
+          if (p.idx32) p.idx32[o] = be;
+        }
+      }
+      // weights: renormalised scores, then the optional dynamic threshold
+      // (the leader stays; the kept shares are renormalised to sum to one)
+      float ksum = 0.f;
+      if (valid && p.dyn_threshold > 0.f) {
+        for (int k = 0; k < p.K; ++k) {
+          const float sh = tmpw[static_cast<size_t>(t) * p.K + k] / psum;
+          if (k == 0 || sh >= p.dyn_threshold) ksum += sh;
+        }
+      }
+      if (valid) {
+        const float denom = p.norm ? (psum + 1e-9f) : 1.f;
+        for (int k = 0; k < p.K; ++k) {
+          const size_t o = static_cast<size_t>(t) * p.K + k;
+          const float pk = tmpw[o];
+          const int e = p.idx32 ? p.idx32[o] : static_cast<int>(p.sel64[o]);
+          float w = p.norm ? pk / denom : pk;
+          bool keep = true;
+          if (p.dyn_threshold > 0.f) {
+            const float sh = pk / psum;
+            keep = k == 0 || sh >= p.dyn_threshold;
+            w = keep ? sh / ksum : 0.f;
+          }
+          if (p.wout) p.wout[o] = w;
+          if (p.w32) p.w32[o] = w;
+          if (p.slot_kept) p.slot_kept[o] = keep ? 1 : 0;
+          if (!keep && p.idx32) p.idx32[o] = E;           // dropped: no row
+          if (keep && p.blockcounts) atomicAdd(&hist[e], 1);
+        }
       }
     }
     if (p.blockcounts) {
@@ -344,13 +422,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
       for (int e = 0; e < E; ++e) lrow[e] = 0.f;
-      if (valid)
-        for (int k = 0; k < p.K; ++k) {
-          const size_t o = static_cast<size_t>(t) * p.K + k;
-          const int e = p.idx32 ? p.idx32[o] : static_cast<int>(p.sel64[o]);
-          const float w = p.w32 ? p.w32[o] : p.wout[o];
-          if (e < E) lrow[e] = w;
+      if (valid) {
+        if (p.K <= 8) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (k < p.K) lrow[se[k]] = sw[k];
+        } else {
+          for (int k = 0; k < p.K; ++k) {
+            const size_t o = static_cast<size_t>(t) * p.K + k;
+            const int e = p.idx32 ? p.idx32[o] : static_cast<int>(p.sel64[o]);
+            const float w = p.w32 ? p.w32[o] : p.wout[o];
+            if (e < E) lrow[e] = w;
+          }
         }
+      }
       asm volatile("bar.sync 1, 128;" ::: "memory");
       for (int e = tid; e < E; e += BM) {
         float g = 0.f, c = 0.f;
@@ -365,8 +450,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   }
   __syncwarp();
-  // the other CTAs keep their shared memory until rank 0 has read it
-  if (p.S > 1) cluster_sync_all();
 
   tc_fence_before();
   __syncthreads();
@@ -449,7 +532,9 @@ cudaError_t launch_npad(const RouteArgs& a, cudaStream_t s) {
   const int m_tiles = (a.T + BM - 1) / BM;
   // split D over a cluster when the row tiles alone would leave SMs idle
   int S = 1;
-  while (S < 8 && m_tiles * S * 2 <= num_sms() && S * 2 <= p.num_kb) S *= 2;
+  constexpr int kMaxSlots =
+      Cfg<NPAD>::STAGES * Cfg<NPAD>::STAGE_BYTES / (BM * Cfg<NPAD>::PART_STRIDE * 4);
+  while (S < 8 && m_tiles * S * 2 <= num_sms() && S * 2 <= p.num_kb && S * 2 <= kMaxSlots) S *= 2;
   p.S = S;
   return launch_k(router_tc_kernel<NPAD>, dim3(m_tiles * p.S), dim3(THREADS), smem_bytes<NPAD>(), s,
                   pdl_enabled(), p.S, mx, mw, p);
