@@ -93,25 +93,30 @@ class ClockSampler:
     def __init__(self, device_index: int, period_s: float = 0.01):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period_s
+        self.device_index = device_index
         self._stop = threading.Event()
+        self._ready = threading.Event()
         self.ok = False
-        try:
-            import pynvml as N
-            self.N = N
-            N.nvmlInit()
-            self.h = N.nvmlDeviceGetHandleByIndex(device_index)
-            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
-            self.ok = True
-        except Exception:
-            self.ok = False
         self.t = threading.Thread(target=self._run, daemon=True)
 
     def _run(self):
-        N = self.N
+        # NVML is initialised and queried on this thread only: a driver call
+        # that stalls can then never block the bench itself
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            h = N.nvmlDeviceGetHandleByIndex(self.device_index)
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._ready.set()
+        if not self.ok:
+            return
         while not self._stop.is_set():
             try:
-                self.samples.append(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
-                bits = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM))
+                bits = N.nvmlDeviceGetCurrentClocksEventReasons(h)
                 for attr, name in self.NAMES.items():
                     v = getattr(N, attr, None)
                     if v is not None and bits & v:
@@ -120,15 +125,18 @@ class ClockSampler:
                 pass
             time.sleep(self.period)
 
-    def start(self):
-        if self.ok:
-            self.t.start()
+    def start(self, wait_s: float = 5.0):
+        """Starts sampling; waits at most ``wait_s`` for NVML to come up."""
+        self.t.start()
+        self._ready.wait(wait_s)
 
-    def stop(self) -> dict:
-        if not self.ok:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+    def stop(self, wait_s: float = 2.0) -> dict:
         self._stop.set()
-        self.t.join()
+        self.t.join(wait_s)
+        if self.t.is_alive() or not self.ok:
+            why = "nvml stalled" if self.t.is_alive() else "nvml unavailable"
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [why],
+                    "samples": len(self.samples)}
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
                 "samples": len(self.samples)}
@@ -208,18 +216,48 @@ class Watchdog:
     def __init__(self, dev, stream, limit_s: float):
         self.dev, self.stream, self.limit_s = dev, stream, limit_s
 
+    def wait_event(self, ev, what: str):
+        t0 = time.monotonic()
+        while not ev.query():
+            if time.monotonic() - t0 > self.limit_s:
+                self.fail(what)
+            time.sleep(0.0005)
+
+    def fail(self, what: str):
+        msg = {"error": f"device work of phase '{what}' did not finish within "
+                        f"{self.limit_s:.0f} s"}
+        try:
+            from mixture_experts_ffn_09_b200 import moe
+            word = moe.device_error_peek()
+            msg["device_error_word"] = hex(word)
+            msg["timed_out_in"] = moe.error_sites(word)
+        except Exception as e:   # the report must not hang or raise
+            msg["device_error_word"] = f"unreadable: {e}"
+        print(json.dumps(msg), flush=True)
+        os._exit(3)
+
     def sync(self, what: str):
         import torch
         ev = torch.cuda.Event()
         ev.record(self.stream)
-        t0 = time.monotonic()
-        while not ev.query():
-            if time.monotonic() - t0 > self.limit_s:
-                print(json.dumps({"error": f"device work of phase '{what}' did not finish within "
-                                           f"{self.limit_s:.0f} s"}), flush=True)
-                os._exit(3)
-            time.sleep(0.0005)
+        self.wait_event(ev, what)
         torch.cuda.synchronize(self.dev)
+
+    def run(self, n: int, fn, what: str, chunk: int = 32):
+        """Calls fn() n times, keeping the host at most two chunks of calls
+        ahead of the device, so a stalled kernel is caught here rather than
+        in a launch that blocks on a full queue."""
+        import torch
+        pending = []
+        for i in range(n):
+            fn()
+            if (i + 1) % chunk == 0 or i + 1 == n:
+                ev = torch.cuda.Event()
+                ev.record(self.stream)
+                pending.append((i, ev))
+                if len(pending) > 2:
+                    j, old = pending.pop(0)
+                    self.wait_event(old, f"{what}, step {j}")
 
 
 def dist_env():
@@ -277,7 +315,9 @@ def run_ours(args, w):
     init_dist(world, "nccl")
     build.build()
     moe.set_gemm_mode({"auto": moe.GEMM_AUTO, "1sm": moe.GEMM_1SM, "2sm": moe.GEMM_2SM}[args.gemm])
-    moe.set_pdl(not args.no_pdl)
+    moe.set_pdl(args.pdl)
+    if args.debug_sync_ms > 0:
+        moe.set_debug_sync(args.debug_sync_ms)
     dev = torch.device("cuda", local)
     d = synth.make_inputs(w)
 
@@ -349,8 +389,7 @@ def run_ours(args, w):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for _ in range(args.steps):
-        step()
+    wd.run(args.steps, step, "timed region")
     t1.record(stream)
     wd.sync("timed region")
     clk = clocks.stop()
@@ -364,8 +403,7 @@ def run_ours(args, w):
     # around every kernel on the launching stream (the events sit between
     # the kernels, so this pass is not the headline number)
     moe.profile_enable(True)
-    for _ in range(max(1, min(args.steps, 50))):
-        step()
+    wd.run(max(1, min(args.steps, 50)), step, "per-stage pass")
     wd.sync("per-stage pass")
     stage_ms, calls = moe.profile_read()
     moe.profile_enable(False)
@@ -387,10 +425,13 @@ def run_ours(args, w):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e_steps):
+
+    def e2e_step():
         xd.copy_(xh, non_blocking=True)
         step(xd, out)
         oh.copy_(out, non_blocking=True)
+
+    wd.run(e_steps, e2e_step, "end-to-end region")
     e1.record(stream)
     wd.sync("end-to-end region")
     e_ms, e_tokens_per_s = throughput(e0.elapsed_time(e1), e_steps, w.T, world, dev)
@@ -432,7 +473,7 @@ def run_ours(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded, shapes of the pages' workloads; random-init weights)",
-        "config": dict(workload_config(w, world), gemm=args.gemm, pdl=not args.no_pdl,
+        "config": dict(workload_config(w, world), gemm=args.gemm, pdl=args.pdl,
                        **({"routing": {"score": args.score, "selection_bias_std": args.selection_bias,
                                        "dynamic_threshold": args.dynamic_threshold,
                                        "capacity_factor": args.capacity_factor,
@@ -540,17 +581,36 @@ def main(argv=None):
     ap.add_argument("--capacity-factor", type=float, default=0.0)
     ap.add_argument("--seq-len", type=int, default=0)
     ap.add_argument("--balance", action="store_true", help="also compute the balancing statistics")
-    ap.add_argument("--no-pdl", action="store_true",
-                    help="launch the kernels without programmatic dependent launch")
+    ap.add_argument("--pdl", action="store_true",
+                    help="launch the kernels with programmatic dependent launch (off by default)")
     ap.add_argument("--watchdog", type=float, default=120.0,
                     help="seconds any wait for the device may take before the run is ended")
+    ap.add_argument("--debug-sync-ms", type=int, default=0,
+                    help="wait (bounded) after every kernel and name the one that does not finish; "
+                         "timings are then not meaningful")
+    ap.add_argument("--deadline", type=float, default=900.0,
+                    help="seconds after which the whole run dumps every thread's stack and exits")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
+    # last bound on the run: whatever blocks (a device wait, a driver call),
+    # the process reports where and ends instead of holding the GPU
+    import faulthandler
+    faulthandler.dump_traceback_later(args.deadline, exit=True)
     w = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
-    else:
+        return
+    try:
         run_ours(args, w)
+    except Exception as e:
+        # a kernel may still be running: leave without the normal teardown,
+        # whose device frees would wait for it
+        import traceback
+        traceback.print_exc()
+        print(json.dumps({"error": f"{type(e).__name__}: {e}"}), flush=True)
+        sys.stdout.flush()
+        sys.stderr.flush()
+        os._exit(3)
 
 
 if __name__ == "__main__":

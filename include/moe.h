@@ -274,12 +274,25 @@ MOE_API int moe_set_fused_gather(int on);
 
 /*
  * Whether the kernels of one forward are launched with programmatic
- * dependent launch (on by default): each kernel's set-up (barriers, tensor
- * memory, descriptor prefetch) overlaps the end of the previous kernel, and
- * it waits for that kernel before reading or writing shared buffers.  Same
- * results either way.  Returns the previous setting.
+ * dependent launch (OFF by default): each kernel's set-up (barriers, tensor
+ * memory, descriptor prefetch) then overlaps the end of the previous kernel,
+ * and it waits for that kernel before reading or writing shared buffers.
+ * Same results either way; it saves 0-2% of a forward.  Off by default
+ * because, with it on, back-to-back forwards of the 64-expert fine-grained
+ * layer were seen to stall on B200 (no cause found; none with it off).
+ * Returns the previous setting.
  */
 MOE_API int moe_set_pdl(int on);
+
+/*
+ * Debug-sync mode (process wide, off by default): with timeout_ms > 0,
+ * moe_ffn_forward waits after every kernel it launches, polling for at most
+ * timeout_ms, and returns MOE_ERR_TIMEOUT naming the first kernel that did
+ * not finish (with the device error word) in moe_last_error().  Kernels then
+ * never overlap and each call is synchronous: for locating a stall, not for
+ * timing.  timeout_ms <= 0 turns it off.  Returns the previous setting.
+ */
+MOE_API int moe_set_debug_sync(int timeout_ms);
 
 /* Short English description of a status code (static storage). */
 MOE_API const char* moe_status_string(moe_status_t status);
@@ -293,9 +306,25 @@ MOE_API int moe_abi_version(void);
 /*
  * Synchronises `stream`, then reads and clears the current device's error
  * word, which kernels set when a bounded wait gives up instead of hanging.
- * Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_CUDA.
+ * Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_CUDA; on MOE_ERR_TIMEOUT,
+ * moe_last_error() names the kernels and roles whose waits gave up.
  */
 MOE_API moe_status_t moe_device_status(void* stream);
+
+/*
+ * Reads the current device's error word into *word WITHOUT waiting for any
+ * caller stream (a copy on a private stream), and does not clear it: for a
+ * host watchdog that wants to know, while kernels may still be running,
+ * whether and where a bounded wait has given up.  Bit 0 = a wait timed out;
+ * bits 8.. = the site (router / grouped GEMM / CTA-pair GEMM, each as
+ * producer, MMA issuer or epilogue, then the test probe).  *word is host
+ * memory.  Returns MOE_OK, MOE_ERR_INVALID_ARG (word NULL) or MOE_ERR_CUDA.
+ */
+MOE_API moe_status_t moe_device_error_peek(unsigned int* word);
+
+/* Comma-separated names of the sites set in an error word (static storage
+   of the calling thread, overwritten by the next call). */
+MOE_API const char* moe_error_sites(unsigned int word);
 
 /*
  * Test hook for failure detection: launches one CTA that waits, through the

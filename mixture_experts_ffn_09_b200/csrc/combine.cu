@@ -17,16 +17,9 @@ namespace {
 
 constexpr int kThreads = 128;
 
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
-  const uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __bfloat1622float2(h[i]);
-    v[2 * i] = f.x;
-    v[2 * i + 1] = f.y;
-  }
-}
+// Slots are read in batches of kBatch: all loads of a batch are issued
+// before the first is used, so each thread keeps several rows in flight.
+constexpr int kBatch = 8;
 
 __global__ void __launch_bounds__(kThreads) combine_bf16_kernel(const __nv_bfloat16* __restrict__ Y,
                                                                 const float* __restrict__ w,
@@ -48,13 +41,29 @@ __global__ void __launch_bounds__(kThreads) combine_bf16_kernel(const __nv_bfloa
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    for (int k = 0; k < K; ++k) {
-      if (sp[k] < 0) continue;                 // a dropped slot adds nothing
-      float y[8];
-      load8(Y + static_cast<size_t>(sp[k]) * D + d, y);
-      const float wk = sw[k];
+    for (int k0 = 0; k0 < K; k0 += kBatch) {
+      uint4 q[kBatch];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(wk, y[i], acc[i]);
+      for (int j = 0; j < kBatch; ++j) {
+        const int k = k0 + j;
+        if (k < K && sp[k] >= 0)
+          q[j] = __ldg(reinterpret_cast<const uint4*>(Y + static_cast<size_t>(sp[k]) * D + d));
+      }
+      // accumulate in slot order; a dropped slot adds nothing
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int k = k0 + j;
+        if (k < K && sp[k] >= 0) {
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q[j]);
+          const float wk = sw[k];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(h[i]);
+            acc[2 * i] = fmaf(wk, f.x, acc[2 * i]);
+            acc[2 * i + 1] = fmaf(wk, f.y, acc[2 * i + 1]);
+          }
+        }
+      }
     }
     uint4 o;
     __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
@@ -81,8 +90,19 @@ __global__ void __launch_bounds__(kThreads) combine_f32_kernel(const float* __re
   const int d_hi = min(D, static_cast<int>(blockIdx.y + 1) * kThreads * 8);
   for (int d = blockIdx.y * kThreads * 8 + threadIdx.x; d < d_hi; d += kThreads) {
     float acc = 0.f;
-    for (int k = 0; k < K; ++k)
-      if (sp[k] >= 0) acc = fmaf(sw[k], __ldg(Y + static_cast<size_t>(sp[k]) * D + d), acc);
+    for (int k0 = 0; k0 < K; k0 += kBatch) {
+      float q[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int k = k0 + j;
+        if (k < K && sp[k] >= 0) q[j] = __ldg(Y + static_cast<size_t>(sp[k]) * D + d);
+      }
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int k = k0 + j;
+        if (k < K && sp[k] >= 0) acc = fmaf(sw[k], q[j], acc);
+      }
+    }
     out[static_cast<size_t>(t) * D + d] = acc;
   }
 }

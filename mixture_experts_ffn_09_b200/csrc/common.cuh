@@ -16,8 +16,23 @@ namespace moe {
 // wide, on by default; see moe_set_pdl).
 bool pdl_enabled();
 
-// Error bits a kernel ORs into the per-device error word.
-enum : unsigned int { DEVERR_TIMEOUT = 1u, DEVERR_BOUNDS = 2u };
+// Error bits a kernel ORs into the per-device error word.  A timed-out
+// wait also sets the bit of its site (kernel and role), so the host can say
+// where a stall happened.
+enum : unsigned int {
+  DEVERR_TIMEOUT = 1u,
+  DEVERR_BOUNDS = 2u,
+  SITE_ROUTER_PRODUCER = 1u << 8,
+  SITE_ROUTER_MMA = 1u << 9,
+  SITE_ROUTER_EPILOGUE = 1u << 10,
+  SITE_GEMM_PRODUCER = 1u << 11,
+  SITE_GEMM_MMA = 1u << 12,
+  SITE_GEMM_EPILOGUE = 1u << 13,
+  SITE_PAIR_PRODUCER = 1u << 14,
+  SITE_PAIR_MMA = 1u << 15,
+  SITE_PAIR_EPILOGUE = 1u << 16,
+  SITE_PROBE = 1u << 17,
+};
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
@@ -120,9 +135,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Waits for the phase of `bar` with the given parity to complete.  Gives up
 // (returns false) when another role of the CTA has already given up
 // (*abort != 0) or after kWaitTimeoutNs, in which case it records the
-// timeout in the device error word and raises *abort for the whole CTA.
+// timeout and its site in the device error word and raises *abort for the
+// whole CTA.  Lanes of one warp can return different results; a caller that
+// goes on to a warp-collective instruction makes the result warp-uniform.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          unsigned int* err,
+                                          unsigned int* err, unsigned int site,
                                           unsigned long long timeout_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
@@ -132,7 +149,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       if (*abort) return false;
       if (globaltimer() - t0 > timeout_ns) {
         *abort = 1;
-        atomicOr(err, DEVERR_TIMEOUT);
+        atomicOr(err, DEVERR_TIMEOUT | site);
         return false;
       }
     }

@@ -100,9 +100,10 @@ __device__ __forceinline__ void decode_tile(const Tail* st, int E, int t, int& e
 
 // Bounded wait that ignores the abort flag: used only on the way out, to let
 // copies and MMAs already in flight land before the CTA leaves.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned int* err) {
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned int* err,
+                                           unsigned int site) {
   int dummy = 0;
-  mbar_wait(bar, parity, &dummy, err);
+  mbar_wait(bar, parity, &dummy, err, site);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -233,7 +234,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int kb = 0; kb < p.num_kb; ++kb) {
         int good = 1;
         if (lane == 0) {
-          good = mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err) ? 1 : 0;
+          good = mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err, SITE_GEMM_PRODUCER) ? 1 : 0;
           if (good) mbar_arrive_expect_tx(&st->full[stage], STAGE_BYTES);
         }
         if (!__shfl_sync(0xffffffffu, good, 0)) { ok = false; break; }
@@ -254,7 +255,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // let every issued load land before the CTA can leave
     if (lane == 0)
       for (int s = 0; s < STAGES; ++s)
-        if (used & (1u << s)) drain_wait(&st->full[s], (last_parity >> s) & 1u, p.err);
+        if (used & (1u << s)) drain_wait(&st->full[s], (last_parity >> s) & 1u, p.err, SITE_GEMM_PRODUCER);
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
@@ -265,12 +266,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
         const int acc = i & 1;
         const uint32_t aph = (i >> 1) & 1;
-        if (!mbar_wait(&st->tempty[acc], aph ^ 1u, abort, p.err)) break;
+        if (!mbar_wait(&st->tempty[acc], aph ^ 1u, abort, p.err, SITE_GEMM_MMA)) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * BN_MMA;
         bool ok = true;
         for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&st->full[stage], phase, abort, p.err)) { ok = false; break; }
+          if (!mbar_wait(&st->full[stage], phase, abort, p.err, SITE_GEMM_MMA)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
@@ -286,7 +287,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       // all MMAs issued by this thread complete before TMEM / smem go away
       umma_commit(&st->mma_done);
-      drain_wait(&st->mma_done, 0, p.err);
+      drain_wait(&st->mma_done, 0, p.err, SITE_GEMM_MMA);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -297,7 +298,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       decode_tile(st, E, t, e, m_blk, n_blk);
       const int acc = i & 1;
       const uint32_t aph = (i >> 1) & 1;
-      if (!mbar_wait(&st->tfull[acc], aph, abort, p.err)) break;
+      // every lane must agree before the warp-collective TMEM loads
+      const bool got = mbar_wait(&st->tfull[acc], aph, abort, p.err, SITE_GEMM_EPILOGUE);
+      if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const int grow = st->off[e] + m_blk * BM + lane_base + lane;
       const bool rvalid = grow < st->off[e + 1];

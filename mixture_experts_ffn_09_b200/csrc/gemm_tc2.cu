@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int kb = 0; kb < p.num_kb; ++kb) {
         int good = 1;
         if (lane == 0) {
-          good = mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err) ? 1 : 0;
+          good = mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err, SITE_PAIR_PRODUCER) ? 1 : 0;
           if (good && leader) mbar_arrive_expect_tx(&st->full[stage], 2 * STAGE_BYTES);
         }
         if (!__shfl_sync(0xffffffffu, good, 0)) { ok = false; break; }
@@ -302,8 +302,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int s = 0; s < STAGES; ++s)
         if (used & (1u << s)) {
           const uint32_t par = (last_parity >> s) & 1u;
-          if (leader) mbar_wait(&st->full[s], par, &dummy, p.err);
-          else mbar_wait(&st->empty[s], par, &dummy, p.err);
+          if (leader) mbar_wait(&st->full[s], par, &dummy, p.err, SITE_PAIR_PRODUCER);
+          else mbar_wait(&st->empty[s], par, &dummy, p.err, SITE_PAIR_PRODUCER);
         }
     }
   } else if (warp == 1) {
@@ -316,12 +316,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int t = cluster_id; t < total; t += num_clusters, ++i) {
         const int acc = i & 1;
         const uint32_t aph = (i >> 1) & 1;
-        if (!mbar_wait(&st->tempty[acc], aph ^ 1u, abort, p.err)) break;
+        if (!mbar_wait(&st->tempty[acc], aph ^ 1u, abort, p.err, SITE_PAIR_MMA)) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * BN_MMA;
         bool ok = true;
         for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&st->full[stage], phase, abort, p.err)) { ok = false; break; }
+          if (!mbar_wait(&st->full[stage], phase, abort, p.err, SITE_PAIR_MMA)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       umma_commit_pair(&st->mma_done);
       int dummy = 0;
-      mbar_wait(&st->mma_done, 0, &dummy, p.err);
+      mbar_wait(&st->mma_done, 0, &dummy, p.err, SITE_PAIR_MMA);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -350,7 +350,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       decode_tile(st, E, t, e, m_blk, n_blk);
       const int acc = i & 1;
       const uint32_t aph = (i >> 1) & 1;
-      if (!mbar_wait(&st->tfull[acc], aph, abort, p.err)) break;
+      // every lane must agree before the warp-collective TMEM loads
+      const bool got = mbar_wait(&st->tfull[acc], aph, abort, p.err, SITE_PAIR_EPILOGUE);
+      if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const int grow = st->off[e] + m_blk * BMP + static_cast<int>(rank) * BMC + lane_base + lane;
       const bool rvalid = grow < st->off[e + 1];

@@ -13,6 +13,8 @@
 #include <string.h>
 
 #include <atomic>
+#include <chrono>
+#include <thread>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -26,7 +28,8 @@ thread_local std::string g_last_error;
 
 std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
 std::atomic<int> g_fused_gather{0};
-std::atomic<int> g_pdl{1};
+std::atomic<int> g_pdl{0};   // programmatic dependent launch: opt-in
+std::atomic<int> g_debug_sync_ms{0};   // > 0: bounded wait after every kernel of a forward
 
 // The tensor-core GEMM for one launch: CTA pairs pay off when experts have
 // enough rows to fill 256-row tiles.  With gather_perm the A rows are read
@@ -72,6 +75,11 @@ struct DevInfo {
   int sms = 0;
   int major = 0, minor = 0;
   unsigned int* err = nullptr;
+  // created once, so that reading the error word during a stall needs no
+  // call that could wait for the device
+  cudaStream_t peek_stream = nullptr;
+  unsigned int* peek_host = nullptr;
+  cudaEvent_t dbg_event = nullptr;
 };
 std::mutex g_dev_mu;
 DevInfo g_dev[64];
@@ -94,6 +102,10 @@ moe_status_t device_info(DevInfo** out) {
     if ((e = cudaGetSymbolAddress(&p, g_device_error)) != cudaSuccess)
       return cuda_fail(e, "cudaGetSymbolAddress(error word)");
     d.err = static_cast<unsigned int*>(p);
+    if ((e = cudaStreamCreateWithFlags(&d.peek_stream, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaMallocHost(&d.peek_host, sizeof(unsigned int))) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&d.dbg_event, cudaEventDisableTiming)) != cudaSuccess)
+      return cuda_fail(e, "device bookkeeping");
     d.init = true;
   }
   if (d.major != 10 || d.minor != 0)
@@ -101,6 +113,46 @@ moe_status_t device_info(DevInfo** out) {
                 d.minor);
   *out = &d;
   return MOE_OK;
+}
+
+// Polls until `done()` or `ms` milliseconds have passed.
+template <typename Done>
+bool poll_ms(int ms, Done done) {
+  const auto t0 = std::chrono::steady_clock::now();
+  while (!done()) {
+    if (std::chrono::steady_clock::now() - t0 > std::chrono::milliseconds(ms)) return false;
+    std::this_thread::sleep_for(std::chrono::microseconds(200));
+  }
+  return true;
+}
+
+// Copies the error word to the host on the private stream; false when the
+// copy does not finish within `ms` (the device is not answering).
+bool peek_word(DevInfo* dev, unsigned int* word, int ms) {
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cudaMemcpyAsync(dev->peek_host, dev->err, sizeof(unsigned int), cudaMemcpyDeviceToHost,
+                      dev->peek_stream) != cudaSuccess)
+    return false;
+  if (!poll_ms(ms, [&] { return cudaStreamQuery(dev->peek_stream) != cudaErrorNotReady; }))
+    return false;
+  *word = *dev->peek_host;
+  return true;
+}
+
+// Debug-sync mode: waits, bounded, for the kernels launched so far on `s`.
+// False (with the error set) when they do not finish in time.
+bool debug_wait(DevInfo* dev, cudaStream_t s, const char* stage) {
+  const int ms = g_debug_sync_ms.load();
+  if (ms <= 0) return true;
+  if (cudaEventRecord(dev->dbg_event, s) == cudaSuccess &&
+      poll_ms(ms, [&] { return cudaEventQuery(dev->dbg_event) != cudaErrorNotReady; }))
+    return true;
+  unsigned int word = 0;
+  const bool got = peek_word(dev, &word, 1000);
+  fail(MOE_ERR_TIMEOUT, "%s did not finish within %d ms (device error word %s0x%x: %s)", stage, ms,
+       got ? "" : "unreadable, ", word, got ? moe_error_sites(word) : "");
+  return false;
 }
 
 // --------------------------------------------------------------- profiler
@@ -429,19 +481,27 @@ moe_status_t moe_ffn_forward_ex(const void* x, const void* router, const void* g
     return moe::launch_balance_finalize(bal, parts, E, Ti, balance_out, s);
   });
   if (e != cudaSuccess) return cuda_fail(e, "router launch");
+  if (!debug_wait(dev, s, "router")) return MOE_ERR_TIMEOUT;
   e = timer.run(1, [&] {
     cudaError_t r = cudaSuccess;
     if (cap > 0.f) {
       r = moe::launch_capacity_clamp(bcount, L.B, E, Ti, K, seq_len, cap, s);
       if (r != cudaSuccess) return r;
+      if (!debug_wait(dev, s, "capacity clamp")) return cudaErrorTimeout;
     }
     r = moe::launch_permute_scan(bcount, L.B, E, bbase, totals, s);
     if (r != cudaSuccess) return r;
+    if (!debug_wait(dev, s, "permute scan")) return cudaErrorTimeout;
     r = moe::launch_permute_scatter(idx32, bbase, totals, bcount, Ti, K, E, offsets, perm, pos,
                                     slot_kept, s);
-    if (r != cudaSuccess || fused_gather) return r;
-    return moe::launch_gather_rows(perm, offsets, E, Ti * K, K, x, Di * elem, xperm, s);
+    if (r != cudaSuccess) return r;
+    if (!debug_wait(dev, s, "permute scatter")) return cudaErrorTimeout;
+    if (fused_gather) return r;
+    r = moe::launch_gather_rows(perm, offsets, E, Ti * K, K, x, Di * elem, xperm, s);
+    if (r != cudaSuccess) return r;
+    return debug_wait(dev, s, "row gather") ? cudaSuccess : cudaErrorTimeout;
   });
+  if (e == cudaErrorTimeout) return MOE_ERR_TIMEOUT;
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   if (dt == MOE_BF16) {
     e = timer.run(2, [&] {
@@ -450,11 +510,13 @@ moe_status_t moe_ffn_forward_ex(const void* x, const void* router, const void* g
                               fused_gather ? perm : nullptr);
     });
     if (e != cudaSuccess) return cuda_fail(e, "gate_up launch");
+    if (!debug_wait(dev, s, "gate_up GEMM")) return MOE_ERR_TIMEOUT;
     e = timer.run(3, [&] {
       return launch_gemm_bf16(2, H, L.Rpad, down_proj, offsets, E, Ti, K, Fi, Di, Di, b2, Y,
                               dev->err, s);
     });
     if (e != cudaSuccess) return cuda_fail(e, "down launch");
+    if (!debug_wait(dev, s, "down GEMM")) return MOE_ERR_TIMEOUT;
   } else {
     e = timer.run(2, [&] {
       return moe::launch_gemm_simt_f32(gu_act, static_cast<const float*>(xperm),
@@ -474,6 +536,7 @@ moe_status_t moe_ffn_forward_ex(const void* x, const void* router, const void* g
                                s);
   });
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  if (!debug_wait(dev, s, "combine")) return MOE_ERR_TIMEOUT;
   return MOE_OK;
 }
 
@@ -490,6 +553,34 @@ moe_status_t moe_debug_bounded_wait(int timeout_ms, void* stream) {
   return MOE_OK;
 }
 
+const char* moe_error_sites(unsigned int word) {
+  static const char* const kNames[] = {"router producer", "router mma", "router epilogue",
+                                       "gemm producer", "gemm mma", "gemm epilogue",
+                                       "pair gemm producer", "pair gemm mma",
+                                       "pair gemm epilogue", "bounded-wait probe"};
+  thread_local std::string out;
+  out.clear();
+  for (int b = 0; b < static_cast<int>(sizeof(kNames) / sizeof(kNames[0])); ++b)
+    if (word & (1u << (8 + b))) {
+      if (!out.empty()) out += ", ";
+      out += kNames[b];
+    }
+  return out.c_str();
+}
+
+moe_status_t moe_device_error_peek(unsigned int* word) {
+  g_last_error.clear();
+  if (!word) return fail(MOE_ERR_INVALID_ARG, "word is NULL");
+  DevInfo* dev = nullptr;
+  moe_status_t st = device_info(&dev);
+  if (st != MOE_OK) return st;
+  if (!peek_word(dev, word, 1000))
+    return fail(MOE_ERR_TIMEOUT, "the device did not answer a 4-byte copy within 1 s");
+  return MOE_OK;
+}
+
+int moe_set_debug_sync(int timeout_ms) { return g_debug_sync_ms.exchange(timeout_ms > 0 ? timeout_ms : 0); }
+
 moe_status_t moe_device_status(void* stream) {
   g_last_error.clear();
   DevInfo* dev = nullptr;
@@ -503,7 +594,8 @@ moe_status_t moe_device_status(void* stream) {
   if (word != 0) {
     const unsigned int zero = 0;
     cudaMemcpy(dev->err, &zero, sizeof zero, cudaMemcpyHostToDevice);
-    return fail(MOE_ERR_TIMEOUT, "device error word 0x%x (1 = a bounded wait timed out)", word);
+    return fail(MOE_ERR_TIMEOUT, "device error word 0x%x (1 = a bounded wait timed out; in: %s)",
+                word, moe_error_sites(word));
   }
   return MOE_OK;
 }

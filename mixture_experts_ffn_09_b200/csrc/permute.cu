@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
 }
 
 constexpr int kGatherThreads = 256;
+constexpr int kGatherBatch = 8;   // 16-byte loads each lane has in flight
 
 __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const int* __restrict__ perm,
                                                                      const int* __restrict__ offsets,
@@ -160,9 +161,24 @@ __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const int* 
   const uint8_t* src = x + static_cast<size_t>(t) * row_bytes;
   uint8_t* dst = x_perm + static_cast<size_t>(r) * row_bytes;
   if ((row_bytes & 15) == 0) {
+    // a batch of independent loads per lane before the stores: enough bytes
+    // in flight per SM to stream at HBM rate
     const uint4* s4 = reinterpret_cast<const uint4*>(src);
     uint4* d4 = reinterpret_cast<uint4*>(dst);
-    for (int i = lane; i < row_bytes / 16; i += 32) d4[i] = __ldg(s4 + i);
+    const int n16 = row_bytes >> 4;
+    for (int i0 = 0; i0 < n16; i0 += 32 * kGatherBatch) {
+      uint4 v[kGatherBatch];
+#pragma unroll
+      for (int j = 0; j < kGatherBatch; ++j) {
+        const int i = i0 + j * 32 + lane;
+        if (i < n16) v[j] = __ldg(s4 + i);
+      }
+#pragma unroll
+      for (int j = 0; j < kGatherBatch; ++j) {
+        const int i = i0 + j * 32 + lane;
+        if (i < n16) d4[i] = v[j];
+      }
+    }
   } else {
     for (int i = lane; i < row_bytes / 4; i += 32)
       reinterpret_cast<uint32_t*>(dst)[i] = reinterpret_cast<const uint32_t*>(src)[i];

@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, used = 0, last_parity = 0;
       for (int kb = kb_lo; kb < kb_hi; ++kb) {
-        if (!mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err)) break;
+        if (!mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err, SITE_ROUTER_PRODUCER)) break;
         mbar_arrive_expect_tx(&st->full[stage], C::STAGE_BYTES);
         tma_load_2d(&tmX, &st->full[stage], sA + stage * A_BYTES, kb * BK, m0);
         tma_load_2d(&tmW, &st->full[stage], sB + stage * C::B_BYTES, kb * BK, 0);
@@ -172,7 +172,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       int dummy = 0;
       for (int s = 0; s < C::STAGES; ++s)
-        if (used & (1u << s)) mbar_wait(&st->full[s], (last_parity >> s) & 1u, &dummy, p.err);
+        if (used & (1u << s))
+          mbar_wait(&st->full[s], (last_parity >> s) & 1u, &dummy, p.err, SITE_ROUTER_PRODUCER);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int kb = kb_lo; kb < kb_hi; ++kb) {
-        if (!mbar_wait(&st->full[stage], phase, abort, p.err)) { ok = false; break; }
+        if (!mbar_wait(&st->full[stage], phase, abort, p.err, SITE_ROUTER_MMA)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
         const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
@@ -195,7 +196,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (ok) umma_commit(&st->tfull);
       umma_commit(&st->mma_done);
       int dummy = 0;
-      mbar_wait(&st->mma_done, 0, &dummy, p.err);
+      mbar_wait(&st->mma_done, 0, &dummy, p.err, SITE_ROUTER_MMA);
     }
   }
   // Partial logits of this CTA's k-blocks: the epilogue warps wait for the
@@ -208,7 +209,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int row = wq * 32 + lane;
   bool have = false;
   if (warp >= 2) {
-    have = mbar_wait(&st->tfull, 0, abort, p.err);
+    // warp-uniform: the TMEM loads below are warp-collective
+    have = __all_sync(0xffffffffu, mbar_wait(&st->tfull, 0, abort, p.err, SITE_ROUTER_EPILOGUE));
     if (have) {
       tc_fence_after();
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

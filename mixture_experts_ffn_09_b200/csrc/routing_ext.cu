@@ -109,7 +109,7 @@ __global__ void bounded_wait_probe_kernel(unsigned long long timeout_ns, unsigne
     mbar_fence_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort, err, timeout_ns);
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort, err, SITE_PROBE, timeout_ns);
   __syncthreads();
 }
 

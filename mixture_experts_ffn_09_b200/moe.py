@@ -103,6 +103,10 @@ def lib() -> ctypes.CDLL:
         L.moe_abi_version.restype = i32
         L.moe_device_status.argtypes = [vp]
         L.moe_device_status.restype = i32
+        L.moe_device_error_peek.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+        L.moe_device_error_peek.restype = i32
+        L.moe_error_sites.argtypes = [ctypes.c_uint]
+        L.moe_error_sites.restype = ctypes.c_char_p
         L.moe_profile_enable.argtypes = [i32]
         L.moe_profile_enable.restype = i32
         L.moe_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), i32]
@@ -111,6 +115,8 @@ def lib() -> ctypes.CDLL:
         L.moe_debug_bounded_wait.restype = i32
         L.moe_set_pdl.argtypes = [i32]
         L.moe_set_pdl.restype = i32
+        L.moe_set_debug_sync.argtypes = [i32]
+        L.moe_set_debug_sync.restype = i32
         L.moe_set_fused_gather.argtypes = [i32]
         L.moe_set_fused_gather.restype = i32
         L.moe_set_gemm_mode.argtypes = [i32]
@@ -388,6 +394,26 @@ def set_fused_gather(on: bool) -> bool:
 def device_status(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device status."""
     return int(lib().moe_device_status(_stream(stream)))
+
+
+def set_debug_sync(timeout_ms: int) -> int:
+    """With timeout_ms > 0 every forward waits, bounded, after each kernel
+    and fails naming the first kernel that did not finish; returns the
+    previous setting."""
+    return int(lib().moe_set_debug_sync(int(timeout_ms)))
+
+
+def device_error_peek() -> int:
+    """The device error word, read without waiting for any stream and
+    without clearing it (for watchdogs)."""
+    w = ctypes.c_uint(0)
+    _check(lib().moe_device_error_peek(ctypes.byref(w)))
+    return int(w.value)
+
+
+def error_sites(word: int) -> str:
+    """Names of the kernel roles whose bounded waits set bits in ``word``."""
+    return lib().moe_error_sites(ctypes.c_uint(word)).decode()
 
 
 def debug_bounded_wait(timeout_ms: int, stream=None) -> None:

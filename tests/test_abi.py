@@ -153,3 +153,12 @@ def test_route_opts_rejected_on_host(L):
     opts = moe._opts(capacity_factor=1.0)
     assert L.moe_route_ex(P, P, None, 64, 64, 8, 2, 1, 0, None, P, P, ctypes.byref(opts),
                           None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_error_sites_decode_on_host(L):
+    """The site bits of the device error word name kernel roles."""
+    assert moe.error_sites(0) == ""
+    assert moe.error_sites(1) == ""
+    assert moe.error_sites(1 | (1 << 16)) == "pair gemm epilogue"
+    assert moe.error_sites((1 << 8) | (1 << 17)) == "router producer, bounded-wait probe"
+    assert L.moe_device_error_peek(None) == moe.MOE_ERR_INVALID_ARG

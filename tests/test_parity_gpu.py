@@ -157,6 +157,32 @@ def test_shapes_and_edges(T, D, F, E, K, act, dtype, gemm_mode):
     _full_check(d, E, K, True, act, dtype)
 
 
+# rows per expert around every tile boundary: 128-row tiles (one CTA) and
+# 256-row pair tiles, whose last tile runs at M = 128 when it holds <= 128 rows
+TAIL_COUNTS = [1, 64, 65, 127, 128, 129, 255, 256, 257, 383, 384, 385]
+
+
+@pytest.mark.parametrize("gemm_mode", MODES, indirect=True)
+@pytest.mark.parametrize("act", ["silu_gated", "relu"])
+def test_tile_tails_every_boundary(act, gemm_mode):
+    """Token t is steered to a chosen expert (a dominant router column), so
+    every expert gets one of TAIL_COUNTS rows; each tile shape and tail is
+    then compared with the oracle on every token."""
+    E, D, F = len(TAIL_COUNTS), 128, 192
+    T = sum(TAIL_COUNTS)
+    d = dict(synth.random_case(77, T, D, F, E, act=act, dtype="bf16", weight_std=0.05))
+    rng = np.random.default_rng(78)
+    owner = rng.permutation(np.repeat(np.arange(E), TAIL_COUNTS))
+    x = rng.standard_normal((T, D), dtype=np.float32) * np.float32(0.1)
+    x[np.arange(T), owner] += np.float32(2.0)
+    router = rng.standard_normal((E, D), dtype=np.float32) * np.float32(0.01)
+    router[np.arange(E), np.arange(E)] = np.float32(8.0)
+    d["x"] = synth.f32_to_bf16_bits(x)
+    d["router"] = synth.f32_to_bf16_bits(router)
+    g, _ = _full_check(d, E, 1, True, act, "bf16")
+    np.testing.assert_array_equal(g["sel"][:, 0], owner)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_norm_topk_prob_off(dtype):
     d = synth.random_case(7, 96, 64, 64, 6, dtype=dtype, weight_std=0.2)
@@ -280,12 +306,18 @@ def test_bounded_wait_times_out_and_the_context_survives():
     the timeout (and is cleared), and a forward afterwards is correct."""
     import time
     from mixture_experts_ffn_09_b200 import moe
+    import torch
     assert moe.device_status() == moe.MOE_OK
     t0 = time.perf_counter()
     moe.debug_bounded_wait(50)
+    torch.cuda.synchronize()
+    word = moe.device_error_peek()                 # seen without clearing it
+    assert word & 1 and "bounded-wait probe" in moe.error_sites(word)
     assert moe.device_status() == moe.MOE_ERR_TIMEOUT
+    assert "bounded-wait probe" in moe.last_error()
     assert time.perf_counter() - t0 < 10.0
     assert moe.device_status() == moe.MOE_OK       # the word was cleared
+    assert moe.device_error_peek() == 0
     w = synth.SILU_SMALL
     _full_check(synth.make_inputs(w), w.E, w.K, w.norm_topk_prob, w.act, w.dtype)
 
