@@ -67,10 +67,11 @@ cudaError_t launch_permute_scatter(const int* idx32, const int* blockbase, const
                                    const int* blockcounts, int T, int K, int E, int* offsets,
                                    int* perm, int* pos, uint8_t* slot_kept, cudaStream_t s);
 
-// x_perm[row, :] = x[perm[row] / K, :] for the sorted rows (at most
-// R_max = T*K; the live count is offsets[E]).
-cudaError_t launch_gather_rows(const int* perm, const int* offsets, int E, int R_max, int K,
-                               const void* x, int row_bytes, void* x_perm, cudaStream_t s);
+// x_perm[pos[t, k], :] = x[t, :] for every slot that was given a row
+// (pos >= 0; perm is the inverse map, offsets[E] the live row count): by
+// sorted row while x fits in L2, else by token with each row of x read once.
+cudaError_t launch_gather_rows(const int* perm, const int* offsets, const int* pos, int T, int E,
+                               int K, const void* x, int row_bytes, void* x_perm, cudaStream_t s);
 
 // out[t, :] = sum_k w[t, k] * Y[pos[t, k], :], fp32 sum in k order; slots
 // with pos < 0 (dropped) add nothing.

@@ -497,7 +497,7 @@ moe_status_t moe_ffn_forward_ex(const void* x, const void* router, const void* g
     if (r != cudaSuccess) return r;
     if (!debug_wait(dev, s, "permute scatter")) return cudaErrorTimeout;
     if (fused_gather) return r;
-    r = moe::launch_gather_rows(perm, offsets, E, Ti * K, K, x, Di * elem, xperm, s);
+    r = moe::launch_gather_rows(perm, offsets, pos, Ti, E, K, x, Di * elem, xperm, s);
     if (r != cudaSuccess) return r;
     return debug_wait(dev, s, "row gather") ? cudaSuccess : cudaErrorTimeout;
   });

@@ -11,7 +11,9 @@
 //   scatter - one CTA per 32-token block ranks its slots within their
 //             expert (warp match + per-warp counts) and writes perm / pos;
 //             slots the router dropped, or past a capacity, get no row;
-//   gather  - one warp per sorted row copies the token row into x_perm.
+//   gather  - copies the token rows into x_perm: one warp per sorted row
+//             while x fits in L2, else one warp per token, which reads each
+//             row of x once and stores it to all of the token's rows.
 #include "common.cuh"
 #include "internal.h"
 
@@ -144,14 +146,14 @@ __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
 }
 
 constexpr int kGatherThreads = 256;
-constexpr int kGatherBatch = 8;   // 16-byte loads each lane has in flight
+constexpr int kGatherBatch = 8;   // 16-byte vectors each lane holds per chunk of a row
 
-__global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const int* __restrict__ perm,
-                                                                     const int* __restrict__ offsets,
-                                                                     int E, int K,
-                                                                     const uint8_t* __restrict__ x,
-                                                                     int row_bytes,
-                                                                     uint8_t* __restrict__ x_perm) {
+// Row order: one warp per sorted row copies x[perm[row] / K].  Every lane
+// issues its whole batch of loads before its stores.  A row of x chosen by
+// several experts is read once per copy; that is cheap while x sits in L2.
+__global__ void __launch_bounds__(kGatherThreads) gather_by_row_kernel(
+    const int* __restrict__ perm, const int* __restrict__ offsets, int E, int K,
+    const uint8_t* __restrict__ x, int row_bytes, uint8_t* __restrict__ x_perm) {
   pdl_trigger();
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -161,8 +163,6 @@ __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const int* 
   const uint8_t* src = x + static_cast<size_t>(t) * row_bytes;
   uint8_t* dst = x_perm + static_cast<size_t>(r) * row_bytes;
   if ((row_bytes & 15) == 0) {
-    // a batch of independent loads per lane before the stores: enough bytes
-    // in flight per SM to stream at HBM rate
     const uint4* s4 = reinterpret_cast<const uint4*>(src);
     uint4* d4 = reinterpret_cast<uint4*>(dst);
     const int n16 = row_bytes >> 4;
@@ -185,6 +185,55 @@ __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const int* 
   }
 }
 
+// Token order: one warp per token reads its row of x once, a chunk of
+// 32 x kGatherBatch 16-byte vectors at a time, and stores each chunk to
+// every sorted row the token's slots were given (pos; a dropped slot has
+// none).  Each x row leaves HBM once however many experts chose it, which
+// matters once x no longer fits in L2.
+__global__ void __launch_bounds__(kGatherThreads) gather_by_token_kernel(
+    const int* __restrict__ pos, int T, int K, const uint8_t* __restrict__ x, int row_bytes,
+    uint8_t* __restrict__ x_perm) {
+  pdl_trigger();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (kGatherThreads / 32) + warp;
+  if (t >= T) return;
+  const int* tp = pos + static_cast<size_t>(t) * K;
+  const int my_row = lane < K ? tp[lane] : -1;     // slots 0..31, shared by shuffle
+  auto row_of = [&](int k) { return k < 32 ? __shfl_sync(0xffffffffu, my_row, k) : __ldg(tp + k); };
+  const uint8_t* src = x + static_cast<size_t>(t) * row_bytes;
+  if ((row_bytes & 15) == 0) {
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    const int n16 = row_bytes >> 4;
+    for (int i0 = 0; i0 < n16; i0 += 32 * kGatherBatch) {
+      uint4 v[kGatherBatch];
+#pragma unroll
+      for (int j = 0; j < kGatherBatch; ++j) {
+        const int i = i0 + j * 32 + lane;
+        if (i < n16) v[j] = __ldg(s4 + i);
+      }
+      for (int k = 0; k < K; ++k) {
+        const int r = row_of(k);
+        if (r < 0) continue;
+        uint4* d4 = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(r) * row_bytes);
+#pragma unroll
+        for (int j = 0; j < kGatherBatch; ++j) {
+          const int i = i0 + j * 32 + lane;
+          if (i < n16) d4[i] = v[j];
+        }
+      }
+    }
+  } else {
+    for (int k = 0; k < K; ++k) {
+      const int r = row_of(k);
+      if (r < 0) continue;
+      uint32_t* dst = reinterpret_cast<uint32_t*>(x_perm + static_cast<size_t>(r) * row_bytes);
+      for (int i = lane; i < row_bytes / 4; i += 32)
+        dst[i] = reinterpret_cast<const uint32_t*>(src)[i];
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_permute_scan(const int* blockcounts, int B, int E, int* blockbase, int* totals,
@@ -201,12 +250,18 @@ cudaError_t launch_permute_scatter(const int* idx32, const int* blockbase, const
                   idx32, blockbase, totals, blockcounts, T, K, E, offsets, perm, pos, slot_kept);
 }
 
-cudaError_t launch_gather_rows(const int* perm, const int* offsets, int E, int R_max, int K,
-                               const void* x, int row_bytes, void* x_perm, cudaStream_t s) {
-  const int rows_per_cta = kGatherThreads / 32;
-  const int grid = (R_max + rows_per_cta - 1) / rows_per_cta;
-  return launch_k(gather_rows_kernel, dim3(grid), dim3(kGatherThreads), 0, s, pdl_enabled(), 1,
-                  perm, offsets, E, K, static_cast<const uint8_t*>(x), row_bytes,
+cudaError_t launch_gather_rows(const int* perm, const int* offsets, const int* pos, int T, int E,
+                               int K, const void* x, int row_bytes, void* x_perm, cudaStream_t s) {
+  constexpr size_t kL2ResidentBytes = 48u << 20;   // x read per copy while it stays in L2
+  const int warps = kGatherThreads / 32;
+  if (static_cast<size_t>(T) * row_bytes <= kL2ResidentBytes) {
+    const long long rows = static_cast<long long>(T) * K;
+    return launch_k(gather_by_row_kernel, dim3(static_cast<unsigned>((rows + warps - 1) / warps)),
+                    dim3(kGatherThreads), 0, s, pdl_enabled(), 1, perm, offsets, E, K,
+                    static_cast<const uint8_t*>(x), row_bytes, static_cast<uint8_t*>(x_perm));
+  }
+  return launch_k(gather_by_token_kernel, dim3((T + warps - 1) / warps), dim3(kGatherThreads), 0, s,
+                  pdl_enabled(), 1, pos, T, K, static_cast<const uint8_t*>(x), row_bytes,
                   static_cast<uint8_t*>(x_perm));
 }
 

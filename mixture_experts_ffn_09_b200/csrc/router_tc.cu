@@ -40,7 +40,9 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int THREADS = 192;
+constexpr int kSlices = 4;                      // epilogue threads per token
+constexpr int kEpiThreads = kSlices * BM;       // warps 2.. (4 per TMEM lane quadrant)
+constexpr int THREADS = 64 + kEpiThreads;
 constexpr int A_BYTES = BM * BK * 2;
 
 template <int NPAD>
@@ -50,7 +52,11 @@ struct Cfg {
   static constexpr int STAGES = (196 * 1024 / STAGE_BYTES) > 12 ? 12 : (196 * 1024 / STAGE_BYTES);
   static constexpr uint32_t TMEM_COLS = NPAD < 32 ? 32 : NPAD;
   static constexpr int PART_STRIDE = NPAD + 1;   // padded rows: conflict-free column access
-  static_assert(BM * PART_STRIDE * 4 <= STAGES * STAGE_BYTES, "partials must fit the ring");
+  // after the partial logits: the slices' maxima and sums, then their
+  // candidate lists (value and index, 8 each)
+  static constexpr int SCRATCH_BYTES = (2 * kSlices * BM + 2 * kSlices * 8 * BM) * 4;
+  static_assert(BM * PART_STRIDE * 4 + SCRATCH_BYTES <= STAGES * STAGE_BYTES,
+                "partials and scratch must fit the ring");
 };
 
 struct Params {
@@ -199,16 +205,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_wait(&st->mma_done, 0, &dummy, p.err, SITE_ROUTER_MMA);
     }
   }
-  // Partial logits of this CTA's k-blocks: the epilogue warps wait for the
-  // MMAs; once every CTA of the cluster is past its MMAs (barrier A, taken
-  // by all threads, so rank 0's ring is free) they store the partials into
-  // slot `rank` of rank 0's shared memory - remote stores for the other
-  // ranks, which do not stall the issuing thread - and barrier B publishes
-  // them to rank 0.
+  // Partial logits of this CTA's k-blocks: warps 2..5 (one per TMEM lane
+  // quadrant) wait for the MMAs; once every CTA of the cluster is past its
+  // MMAs (barrier A, taken by all threads, so rank 0's ring is free) they
+  // store the partials of the valid token rows into slot `rank` of rank 0's
+  // shared memory - remote stores for the other ranks - and barrier B
+  // publishes them to rank 0.
   const int wq = warp & 3;
   const int row = wq * 32 + lane;
+  const int slice = warp >= 2 ? (warp - 2) >> 2 : 0;   // which quarter of the experts
+  const int t = m0 + row;
+  const bool valid = t < p.T;
   bool have = false;
-  if (warp >= 2) {
+  if (warp >= 2 && slice == 0) {
     // warp-uniform: the TMEM loads below are warp-collective
     have = __all_sync(0xffffffffu, mbar_wait(&st->tfull, 0, abort, p.err, SITE_ROUTER_EPILOGUE));
     if (have) {
@@ -225,6 +234,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t r[32];
       tmem_ld32(tb + c0, r);
       tmem_ld_wait();
+      if (!valid) continue;                 // padding rows: nothing to reduce
       if (rank == 0) {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
@@ -241,29 +251,44 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (p.S > 1) cluster_sync_all(); else __syncthreads();            // B
 
   if (warp >= 2 && rank == 0 && !*abort) {
-    // ------------------------------------------------ one token per thread
-    const int t = m0 + row;
-    const bool valid = t < p.T;
+    // ------------------------------------------- kSlices threads per token
+    // Thread `slice` of a token owns experts [e_lo, e_hi); the 16 epilogue
+    // warps meet at named barrier 1.  The row's logits live in lrow
+    // (shared memory), updated in place by the slice owners.
+    auto epi_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); };
     int* hist = st->hist[wq];
     float* lrow = part + row * C::PART_STRIDE;
-    // sum the split partials in rank order (all local now)
-    for (int q = 1; q < p.S; ++q) {
-      const float* src = part + (q * BM + row) * C::PART_STRIDE;
-      for (int e = 0; e < E; ++e) lrow[e] += src[e];
-    }
-    // add the bias, write the logits
-    float m = -INFINITY;
-    for (int e = 0; e < E; ++e) {
+    float* red = part + p.S * BM * C::PART_STRIDE;           // [2][kSlices][BM]
+    float* cand_v = red + 2 * kSlices * BM;                  // [kSlices][8][BM]
+    int* cand_e = reinterpret_cast<int*>(cand_v + kSlices * 8 * BM);
+    constexpr int CW = NPAD / kSlices;
+    const int e_lo = slice * CW;
+    const int e_hi = min(E, e_lo + CW);
+    // sum the split partials in rank order, add the bias, write the logits
+    float lmax = -INFINITY;
+    for (int e = e_lo; e < e_hi; ++e) {
       float v = lrow[e];
+      for (int q = 1; q < p.S; ++q) v += part[(q * BM + row) * C::PART_STRIDE + e];
       if (p.bias) v += __ldg(p.bias + e);
       if (valid && p.logits) p.logits[static_cast<size_t>(t) * E + e] = v;
       if (isnan(v)) v = -INFINITY;
       lrow[e] = v;
-      m = fmaxf(m, v);
+      lmax = fmaxf(lmax, v);
     }
+    red[slice * BM + row] = lmax;
+    epi_sync();
+    float m = red[row];
+#pragma unroll
+    for (int j = 1; j < kSlices; ++j) m = fmaxf(m, red[j * BM + row]);
     float s = 0.f;
-    if (p.score == 0)
-      for (int e = 0; e < E; ++e) s += expf(lrow[e] - m);
+    if (p.score == 0) {
+      float ls = 0.f;
+      for (int e = e_lo; e < e_hi; ++e) ls += expf(lrow[e] - m);
+      red[(kSlices + slice) * BM + row] = ls;
+      epi_sync();
+#pragma unroll
+      for (int j = 0; j < kSlices; ++j) s += red[(kSlices + j) * BM + row];   // fixed order
+    }
     // score of expert e: softmax probability or sigmoid of the logit
     auto score = [&](int e) {
       const float l = lrow[e];
@@ -272,15 +297,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ranking key: the logit (monotone in either score) unless a selection
     // bias is added to the score
     auto key = [&](int e) { return p.sel_bias ? score(e) + __ldg(p.sel_bias + e) : lrow[e]; };
-    // K rounds of selection, then the weights.  For K <= 8 the choices stay
-    // in registers; larger K parks them in the output buffers between the
-    // two loops.
     int se[8];
     float sw[8];
+    bool kp[8];
     if (p.K <= 8) {
-      // one pass over the experts, bubbling each into a sorted list of the
-      // best K (value descending, index ascending: a later equal value never
-      // overtakes, so the lower index stays ahead)
+      // each slice keeps a sorted list of its best K (value descending,
+      // index ascending: a later equal value never overtakes, so the lower
+      // index stays ahead); thread 0 of the token merges the lists, whose
+      // index ranges are disjoint and ascending in slice order
       float tv[8];
       int te[8];
 #pragma unroll
@@ -288,7 +312,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tv[k] = -INFINITY;
         te[k] = 0x7fffffff;
       }
-      for (int e = 0; e < E; ++e) {
+      for (int e = e_lo; e < e_hi; ++e) {
         float v = key(e);
         int ve = e;
 #pragma unroll
@@ -303,51 +327,90 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      float pk[8];
-      float psum = 0.f;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        if (k < p.K) {
-          se[k] = te[k];
-          pk[k] = score(te[k]);
-          psum += pk[k];
-        }
+        cand_v[(slice * 8 + k) * BM + row] = tv[k];
+        cand_e[(slice * 8 + k) * BM + row] = te[k];
       }
-      float ksum = 0.f;
-      if (p.dyn_threshold > 0.f) {
+      epi_sync();
+      if (slice == 0) {
+        int head[kSlices];
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
+        for (int j = 0; j < kSlices; ++j) head[j] = 0;
+        float pk[8];
+        float psum = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
           if (k < p.K) {
-            const float sh = pk[k] / psum;
-            if (k == 0 || sh >= p.dyn_threshold) ksum += sh;
-          }
-      }
-      const float denom = p.norm ? (psum + 1e-9f) : 1.f;
+            int bj = 0;
+            float bv = cand_v[(0 * 8 + head[0]) * BM + row];
+            int be = cand_e[(0 * 8 + head[0]) * BM + row];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        if (k < p.K) {
-          float w = p.norm ? pk[k] / denom : pk[k];
-          bool keep = true;
-          if (p.dyn_threshold > 0.f) {
-            const float sh = pk[k] / psum;
-            keep = k == 0 || sh >= p.dyn_threshold;
-            w = keep ? sh / ksum : 0.f;
+            for (int j = 1; j < kSlices; ++j) {
+              const float v = cand_v[(j * 8 + head[j]) * BM + row];
+              const int e = cand_e[(j * 8 + head[j]) * BM + row];
+              if (ranks_before(v, e, bv, be)) {
+                bv = v;
+                be = e;
+                bj = j;
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < kSlices; ++j) head[j] += (j == bj) ? 1 : 0;
+            se[k] = be;
+            pk[k] = score(be);
+            psum += pk[k];
           }
-          sw[k] = w;
-          if (valid) {
-            const size_t o = static_cast<size_t>(t) * p.K + k;
-            if (p.sel64) p.sel64[o] = se[k];
-            if (p.wout) p.wout[o] = w;
-            if (p.w32) p.w32[o] = w;
-            if (p.idx32) p.idx32[o] = keep ? se[k] : E;   // dropped: no row
-            if (p.slot_kept) p.slot_kept[o] = keep ? 1 : 0;
-            if (keep && p.blockcounts) atomicAdd(&hist[se[k]], 1);
+        }
+        float ksum = 0.f;
+        if (p.dyn_threshold > 0.f) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (k < p.K) {
+              const float sh = pk[k] / psum;
+              if (k == 0 || sh >= p.dyn_threshold) ksum += sh;
+            }
+        }
+        const float denom = p.norm ? (psum + 1e-9f) : 1.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (k < p.K) {
+            float w = p.norm ? pk[k] / denom : pk[k];
+            bool keep = true;
+            if (p.dyn_threshold > 0.f) {
+              const float sh = pk[k] / psum;
+              keep = k == 0 || sh >= p.dyn_threshold;
+              w = keep ? sh / ksum : 0.f;
+            }
+            sw[k] = w;
+            kp[k] = keep;
+            if (valid) {
+              const size_t o = static_cast<size_t>(t) * p.K + k;
+              if (p.sel64) p.sel64[o] = se[k];
+              if (p.wout) p.wout[o] = w;
+              if (p.w32) p.w32[o] = w;
+              if (p.idx32) p.idx32[o] = keep ? se[k] : E;   // dropped: no row
+              if (p.slot_kept) p.slot_kept[o] = keep ? 1 : 0;
+            }
+          }
+        }
+        // per-warp expert counts: one shared atomic per distinct expert
+        if (p.blockcounts) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            if (k < p.K) {
+              const int ek = (valid && kp[k]) ? se[k] : -1;
+              const unsigned int same = __match_any_sync(0xffffffffu, ek);
+              if (ek >= 0 && lane == __ffs(same) - 1) atomicAdd(&hist[ek], __popc(same));
+            }
           }
         }
       }
-    } else {
-      // the chosen index goes to sel64 / idx32 and the unbiased score to the
-      // weight buffer until the weights are final
+    } else if (slice == 0) {
+      // K > 8: the k-th choice is the best entry that ranks strictly after
+      // the (k-1)-th, one scan over the row per round; the chosen index goes
+      // to sel64 / idx32 and the unbiased score to the weight buffer until
+      // the weights are final
       float* tmpw = p.w32 ? p.w32 : p.wout;
       float lv = INFINITY;
       int le = -1;
@@ -382,10 +445,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (k == 0 || sh >= p.dyn_threshold) ksum += sh;
         }
       }
-      if (valid) {
-        const float denom = p.norm ? (psum + 1e-9f) : 1.f;
-        for (int k = 0; k < p.K; ++k) {
-          const size_t o = static_cast<size_t>(t) * p.K + k;
+      const float denom = p.norm ? (psum + 1e-9f) : 1.f;
+      for (int k = 0; k < p.K; ++k) {
+        const size_t o = static_cast<size_t>(t) * p.K + k;
+        int ek = -1;
+        if (valid) {
           const float pk = tmpw[o];
           const int e = p.idx32 ? p.idx32[o] : static_cast<int>(p.sel64[o]);
           float w = p.norm ? pk / denom : pk;
@@ -399,30 +463,35 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (p.w32) p.w32[o] = w;
           if (p.slot_kept) p.slot_kept[o] = keep ? 1 : 0;
           if (!keep && p.idx32) p.idx32[o] = E;           // dropped: no row
-          if (keep && p.blockcounts) atomicAdd(&hist[e], 1);
+          if (keep) ek = e;
+        }
+        if (p.blockcounts) {
+          const unsigned int same = __match_any_sync(0xffffffffu, ek);
+          if (ek >= 0 && lane == __ffs(same) - 1) atomicAdd(&hist[ek], __popc(same));
         }
       }
     }
-    if (p.blockcounts) {
+    if (slice == 0 && p.blockcounts) {
       __syncwarp();
       const int b = (m0 + wq * 32) / 32;
       if (m0 + wq * 32 < p.T)
         for (int e = lane; e < E; e += 32) p.blockcounts[static_cast<size_t>(b) * E + e] = hist[e];
     }
-    if (p.bal_partial) {
+    if (slice == 0 && p.bal_partial) {
       // per-tile column sums of the scores, the gate and gate > 0, each in
-      // row order (deterministic); the 128 epilogue threads share barrier 1
+      // row order (deterministic); the 128 threads of slice 0 meet at
+      // named barrier 2
       const int tid = row;
       float* bp = p.bal_partial + static_cast<size_t>(blockIdx.x / p.S) * 3 * E;
       // the row's scores replace its logits (score(e) reads only lrow[e])
       for (int e = 0; e < E; ++e) lrow[e] = valid ? score(e) : 0.f;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 2, 128;" ::: "memory");
       for (int e = tid; e < E; e += BM) {
         float acc = 0.f;
         for (int r = 0; r < BM; ++r) acc += part[r * C::PART_STRIDE + e];
         bp[e] = acc;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 2, 128;" ::: "memory");
       for (int e = 0; e < E; ++e) lrow[e] = 0.f;
       if (valid) {
         if (p.K <= 8) {
@@ -438,7 +507,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 2, 128;" ::: "memory");
       for (int e = tid; e < E; e += BM) {
         float g = 0.f, c = 0.f;
         for (int r = 0; r < BM; ++r) {
@@ -534,8 +603,8 @@ cudaError_t launch_npad(const RouteArgs& a, cudaStream_t s) {
   const int m_tiles = (a.T + BM - 1) / BM;
   // split D over a cluster when the row tiles alone would leave SMs idle
   int S = 1;
-  constexpr int kMaxSlots =
-      Cfg<NPAD>::STAGES * Cfg<NPAD>::STAGE_BYTES / (BM * Cfg<NPAD>::PART_STRIDE * 4);
+  constexpr int kMaxSlots = (Cfg<NPAD>::STAGES * Cfg<NPAD>::STAGE_BYTES - Cfg<NPAD>::SCRATCH_BYTES) /
+                            (BM * Cfg<NPAD>::PART_STRIDE * 4);
   while (S < 8 && m_tiles * S * 2 <= num_sms() && S * 2 <= p.num_kb && S * 2 <= kMaxSlots) S *= 2;
   p.S = S;
   return launch_k(router_tc_kernel<NPAD>, dim3(m_tiles * p.S), dim3(THREADS), smem_bytes<NPAD>(), s,

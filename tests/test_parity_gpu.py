@@ -183,6 +183,13 @@ def test_tile_tails_every_boundary(act, gemm_mode):
     np.testing.assert_array_equal(g["sel"][:, 0], owner)
 
 
+def test_gather_by_token_when_x_exceeds_l2():
+    """x of 64 MB (T=8192, D=4096, bf16) is gathered token by token (each row
+    of x read once); every token is checked against the oracle."""
+    d = synth.random_case(91, 8192, 4096, 64, 4, dtype="bf16", weight_std=0.02)
+    _full_check(d, 4, 2, True, "silu_gated", "bf16")
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_norm_topk_prob_off(dtype):
     d = synth.random_case(7, 96, 64, 64, 6, dtype=dtype, weight_std=0.2)
