@@ -365,3 +365,60 @@ def test_programmatic_dependent_launch_changes_nothing(gemm_mode):
     for a, b in zip(outs[False], outs[True]):
         for k in ("out", "sel", "w", "logits"):
             np.testing.assert_array_equal(a[k], b[k])
+
+
+def test_debug_sync_mode_changes_nothing():
+    """With a bounded wait after every kernel the forward returns the same
+    bits, and the mode switches back off."""
+    from mixture_experts_ffn_09_b200 import moe
+    d = synth.random_case(21, 300, 128, 192, 8, dtype="bf16", weight_std=0.05)
+    dev = PL.to_device(d)
+    a = PL.run_gpu(dev, 8, 2, True, "silu_gated")
+    prev = moe.set_debug_sync(5000)
+    try:
+        b = PL.run_gpu(dev, 8, 2, True, "silu_gated")
+    finally:
+        assert moe.set_debug_sync(prev) == 5000
+    for k in ("out", "sel", "w", "logits"):
+        np.testing.assert_array_equal(a[k], b[k])
+
+
+@pytest.mark.parametrize("gemm_mode", MODES, indirect=True)
+def test_forward_replays_from_a_cuda_graph(gemm_mode):
+    """The forward makes no synchronising call, so it can be captured into a
+    CUDA graph; replays give the eager result bit for bit."""
+    import torch
+    from mixture_experts_ffn_09_b200 import moe
+    d = synth.random_case(22, 640, 256, 384, 8, dtype="bf16", weight_std=0.05)
+    dev = PL.to_device(d)
+    x = dev["x"]
+    T, D = x.shape
+    F = dev["down_proj"].shape[-1]
+    ws = torch.empty(moe.workspace_size(T, D, F, 8, 2, moe.BF16, moe.ACT_SILU_GATED),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(x)
+    sel = torch.empty(T, 2, dtype=torch.int64, device="cuda")
+    w = torch.empty(T, 2, dtype=torch.float32, device="cuda")
+
+    def fwd():
+        moe.ffn_forward(x, dev["router"], dev["gate_up_proj"], dev["down_proj"], 8, 2, True,
+                        moe.ACT_SILU_GATED, out, sel, w, None, None, None, None, ws)
+
+    fwd()                                   # first call sets kernel attributes
+    torch.cuda.synchronize()
+    ref = (out.clone(), sel.clone(), w.clone())
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fwd()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fwd()
+    for _ in range(3):
+        out.zero_()
+        sel.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref[0]) and torch.equal(sel, ref[1]) and torch.equal(w, ref[2])
+    assert moe.device_status() == moe.MOE_OK
