@@ -9,7 +9,9 @@
 // pair stages its own 128 rows of A and HALF of the 256 B rows, and the pair's
 // MMA reads both CTAs' shared memory, so a CTA moves 32 KB per k-block for
 // the same 128 x 256 x 64 product that costs 48 KB on one CTA.  The saved
-// shared memory buys a 6-stage ring.
+// shared memory buys a 7-stage ring (224 KB: the ring starts at the
+// 1024-byte-aligned base of dynamic shared memory, and the tile table keeps
+// only the per-expert tile starts and row offsets).
 //
 // Cluster of 2 CTAs (rank 0 = leader), 192 threads each:
 //   warp 0 (both)   TMA producer for this CTA's A rows and B half; the loads
@@ -40,7 +42,7 @@ constexpr int BMC = 128;                      // rows per CTA
 constexpr int BMP = 256;                      // rows per pair
 constexpr int BK = 64;
 constexpr int BN_MMA = 256;
-constexpr int STAGES = 6;
+constexpr int STAGES = 7;
 constexpr int A_BYTES = BMC * BK * 2;         // 16 KB
 constexpr int B_BYTES = (BN_MMA / 2) * BK * 2;  // 16 KB (this CTA's half)
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -73,11 +75,10 @@ struct Tail {
   int abort;
   int total_tiles;
   int tile_start[kMaxExperts + 1];
-  int mt[kMaxExperts];
   int off[kMaxExperts + 1];
 };
 
-constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(Tail);
+constexpr size_t kSmemBytes = STAGES * STAGE_BYTES + sizeof(Tail);
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -149,8 +150,8 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
       : "memory");
 }
 
-__device__ __forceinline__ void decode_tile(const Tail* st, int E, int t, int& e, int& m_blk,
-                                            int& n_blk) {
+__device__ __forceinline__ void decode_tile(const Tail* st, int E, int n_tiles, int t, int& e,
+                                            int& m_blk, int& n_blk) {
   int lo = 0, hi = E - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -158,7 +159,7 @@ __device__ __forceinline__ void decode_tile(const Tail* st, int E, int t, int& e
   }
   e = lo;
   const int local = t - st->tile_start[e];
-  const int mt = st->mt[e];
+  const int mt = (st->tile_start[e + 1] - st->tile_start[e]) / n_tiles;
   n_blk = local / mt;
   m_blk = local - n_blk * mt;
 }
@@ -185,9 +186,12 @@ template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB, const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
+  if ((smem_u32(smem_raw) & 1023u) != 0) {   // the ring needs 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(p.err, DEVERR_BOUNDS);
+    return;
+  }
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
   Tail* st = reinterpret_cast<Tail*>(smem + STAGES * STAGE_BYTES);
@@ -231,7 +235,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int o0 = p.offsets[e], o1 = p.offsets[e + 1];
       const int mt = (o1 - o0 + BMP - 1) / BMP;
       st->off[e] = o0;
-      st->mt[e] = mt;
       st->tile_start[e] = acc;
       acc += mt * n_tiles;
     }
@@ -259,7 +262,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int t = cluster_id; t < total; t += num_clusters) {
       if (!__shfl_sync(0xffffffffu, lane == 0 ? static_cast<int>(!*abort) : 0, 0)) break;
       int e, m_blk, n_blk;
-      decode_tile(st, E, t, e, m_blk, n_blk);
+      decode_tile(st, E, n_tiles, t, e, m_blk, n_blk);
       const int rowA = st->off[e] + m_blk * BMP + static_cast<int>(rank) * BMC;
       const int rowB = (EPI == kSiluGated)
                            ? e * p.b_rows + n_blk * 128 + (leader ? 0 : p.up_off)
@@ -347,7 +350,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     int i = 0;
     for (int t = cluster_id; t < total; t += num_clusters, ++i) {
       int e, m_blk, n_blk;
-      decode_tile(st, E, t, e, m_blk, n_blk);
+      decode_tile(st, E, n_tiles, t, e, m_blk, n_blk);
       const int acc = i & 1;
       const uint32_t aph = (i >> 1) & 1;
       // every lane must agree before the warp-collective TMEM loads
