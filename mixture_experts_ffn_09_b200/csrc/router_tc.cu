@@ -43,6 +43,7 @@ constexpr int BK = 64;
 constexpr int kSlices = 4;                      // epilogue threads per token
 constexpr int kEpiThreads = kSlices * BM;       // warps 2.. (4 per TMEM lane quadrant)
 constexpr int THREADS = 64 + kEpiThreads;
+constexpr int kDroppedBit = 1 << 30;              // marks a slot the threshold dropped
 constexpr int A_BYTES = BM * BK * 2;
 
 template <int NPAD>
@@ -52,9 +53,9 @@ struct Cfg {
   static constexpr int STAGES = (196 * 1024 / STAGE_BYTES) > 12 ? 12 : (196 * 1024 / STAGE_BYTES);
   static constexpr uint32_t TMEM_COLS = NPAD < 32 ? 32 : NPAD;
   static constexpr int PART_STRIDE = NPAD + 1;   // padded rows: conflict-free column access
-  // after the partial logits: the slices' maxima and sums, then their
-  // candidate lists (value and index, 8 each)
-  static constexpr int SCRATCH_BYTES = (2 * kSlices * BM + 2 * kSlices * 8 * BM) * 4;
+  // after the partial logits: the slices' maxima and sums, their candidate
+  // lists (value and index, 8 each), then the token's final choices
+  static constexpr int SCRATCH_BYTES = (2 * kSlices * BM + 2 * kSlices * 8 * BM + 2 * 8 * BM) * 4;
   static_assert(BM * PART_STRIDE * 4 + SCRATCH_BYTES <= STAGES * STAGE_BYTES,
                 "partials and scratch must fit the ring");
 };
@@ -261,6 +262,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     float* red = part + p.S * BM * C::PART_STRIDE;           // [2][kSlices][BM]
     float* cand_v = red + 2 * kSlices * BM;                  // [kSlices][8][BM]
     int* cand_e = reinterpret_cast<int*>(cand_v + kSlices * 8 * BM);
+    int* sel_e = cand_e + kSlices * 8 * BM;                  // [8][BM] final choices
+    float* sel_p = reinterpret_cast<float*>(sel_e + 8 * BM);  // [8][BM] their weights
     constexpr int CW = NPAD / kSlices;
     const int e_lo = slice * CW;
     const int e_hi = min(E, e_lo + CW);
@@ -297,14 +300,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ranking key: the logit (monotone in either score) unless a selection
     // bias is added to the score
     auto key = [&](int e) { return p.sel_bias ? score(e) + __ldg(p.sel_bias + e) : lrow[e]; };
-    int se[8];
-    float sw[8];
-    bool kp[8];
     if (p.K <= 8) {
-      // each slice keeps a sorted list of its best K (value descending,
-      // index ascending: a later equal value never overtakes, so the lower
-      // index stays ahead); thread 0 of the token merges the lists, whose
-      // index ranges are disjoint and ascending in slice order
+      // each slice keeps a sorted list of its best entries (value
+      // descending, index ascending: a later equal value never overtakes, so
+      // the lower index stays ahead); the list holds 8 and only its first K
+      // are used.  Thread 0 of the token merges the slices' lists, whose
+      // index ranges are disjoint and ascending in slice order.
       float tv[8];
       int te[8];
 #pragma unroll
@@ -313,19 +314,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         te[k] = 0x7fffffff;
       }
       for (int e = e_lo; e < e_hi; ++e) {
-        float v = key(e);
-        int ve = e;
+        // insert e into the sorted list: the list is sorted, so "e ranks
+        // before entry k" holds from some k on; every entry is then a select
+        // from the old list (no chain of dependent swaps)
+        const float v = key(e);
+        bool b[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (k < p.K && ranks_before(v, ve, tv[k], te[k])) {
-            const float sv = tv[k];
-            const int si = te[k];
-            tv[k] = v;
-            te[k] = ve;
-            v = sv;
-            ve = si;
-          }
+        for (int k = 0; k < 8; ++k) b[k] = ranks_before(v, e, tv[k], te[k]);
+#pragma unroll
+        for (int k = 7; k > 0; --k) {
+          tv[k] = b[k] ? (b[k - 1] ? tv[k - 1] : v) : tv[k];
+          te[k] = b[k] ? (b[k - 1] ? te[k - 1] : e) : te[k];
         }
+        tv[0] = b[0] ? v : tv[0];
+        te[0] = b[0] ? e : te[0];
       }
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -334,75 +336,71 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       epi_sync();
       if (slice == 0) {
-        int head[kSlices];
-#pragma unroll
-        for (int j = 0; j < kSlices; ++j) head[j] = 0;
-        float pk[8];
+        // Short rolled loops from here on: each router CTA runs this code
+        // once per launch with a cold instruction cache, so code size costs
+        // more than the few extra shared-memory accesses.  The choices go to
+        // sel_e / sel_p (index, unbiased score; the index's top bit marks a
+        // slot the threshold dropped).
+        int head0 = 0, head1 = 0, head2 = 0, head3 = 0;
         float psum = 0.f;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (k < p.K) {
-            int bj = 0;
-            float bv = cand_v[(0 * 8 + head[0]) * BM + row];
-            int be = cand_e[(0 * 8 + head[0]) * BM + row];
-#pragma unroll
-            for (int j = 1; j < kSlices; ++j) {
-              const float v = cand_v[(j * 8 + head[j]) * BM + row];
-              const int e = cand_e[(j * 8 + head[j]) * BM + row];
-              if (ranks_before(v, e, bv, be)) {
-                bv = v;
-                be = e;
-                bj = j;
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < kSlices; ++j) head[j] += (j == bj) ? 1 : 0;
-            se[k] = be;
-            pk[k] = score(be);
-            psum += pk[k];
-          }
+#pragma unroll 1
+        for (int k = 0; k < p.K; ++k) {
+          float bv = cand_v[(0 * 8 + head0) * BM + row];
+          int be = cand_e[(0 * 8 + head0) * BM + row];
+          int bj = 0;
+          const float v1 = cand_v[(1 * 8 + head1) * BM + row];
+          const int e1 = cand_e[(1 * 8 + head1) * BM + row];
+          if (ranks_before(v1, e1, bv, be)) { bv = v1; be = e1; bj = 1; }
+          const float v2 = cand_v[(2 * 8 + head2) * BM + row];
+          const int e2 = cand_e[(2 * 8 + head2) * BM + row];
+          if (ranks_before(v2, e2, bv, be)) { bv = v2; be = e2; bj = 2; }
+          const float v3 = cand_v[(3 * 8 + head3) * BM + row];
+          const int e3 = cand_e[(3 * 8 + head3) * BM + row];
+          if (ranks_before(v3, e3, bv, be)) { bv = v3; be = e3; bj = 3; }
+          head0 += bj == 0;
+          head1 += bj == 1;
+          head2 += bj == 2;
+          head3 += bj == 3;
+          const float pk = score(be);
+          sel_e[k * BM + row] = be;
+          sel_p[k * BM + row] = pk;
+          psum += pk;
         }
         float ksum = 0.f;
         if (p.dyn_threshold > 0.f) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            if (k < p.K) {
-              const float sh = pk[k] / psum;
-              if (k == 0 || sh >= p.dyn_threshold) ksum += sh;
-            }
-        }
-        const float denom = p.norm ? (psum + 1e-9f) : 1.f;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (k < p.K) {
-            float w = p.norm ? pk[k] / denom : pk[k];
-            bool keep = true;
-            if (p.dyn_threshold > 0.f) {
-              const float sh = pk[k] / psum;
-              keep = k == 0 || sh >= p.dyn_threshold;
-              w = keep ? sh / ksum : 0.f;
-            }
-            sw[k] = w;
-            kp[k] = keep;
-            if (valid) {
-              const size_t o = static_cast<size_t>(t) * p.K + k;
-              if (p.sel64) p.sel64[o] = se[k];
-              if (p.wout) p.wout[o] = w;
-              if (p.w32) p.w32[o] = w;
-              if (p.idx32) p.idx32[o] = keep ? se[k] : E;   // dropped: no row
-              if (p.slot_kept) p.slot_kept[o] = keep ? 1 : 0;
-            }
+#pragma unroll 1
+          for (int k = 0; k < p.K; ++k) {
+            const float sh = sel_p[k * BM + row] / psum;
+            if (k == 0 || sh >= p.dyn_threshold) ksum += sh;
           }
         }
-        // per-warp expert counts: one shared atomic per distinct expert
-        if (p.blockcounts) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            if (k < p.K) {
-              const int ek = (valid && kp[k]) ? se[k] : -1;
-              const unsigned int same = __match_any_sync(0xffffffffu, ek);
-              if (ek >= 0 && lane == __ffs(same) - 1) atomicAdd(&hist[ek], __popc(same));
-            }
+        const float denom = p.norm ? (psum + 1e-9f) : 1.f;
+#pragma unroll 1
+        for (int k = 0; k < p.K; ++k) {
+          const float pk = sel_p[k * BM + row];
+          const int e = sel_e[k * BM + row];
+          float w = p.norm ? pk / denom : pk;
+          bool keep = true;
+          if (p.dyn_threshold > 0.f) {
+            const float sh = pk / psum;
+            keep = k == 0 || sh >= p.dyn_threshold;
+            w = keep ? sh / ksum : 0.f;
+          }
+          sel_p[k * BM + row] = w;                 // the final weight from here on
+          if (!keep) sel_e[k * BM + row] = e | kDroppedBit;
+          if (valid) {
+            const size_t o = static_cast<size_t>(t) * p.K + k;
+            if (p.sel64) p.sel64[o] = e;
+            if (p.wout) p.wout[o] = w;
+            if (p.w32) p.w32[o] = w;
+            if (p.idx32) p.idx32[o] = keep ? e : E;   // dropped: no row
+            if (p.slot_kept) p.slot_kept[o] = keep ? 1 : 0;
+          }
+          // per-warp expert counts: one shared atomic per distinct expert
+          if (p.blockcounts) {
+            const int ek = (valid && keep) ? e : -1;
+            const unsigned int same = __match_any_sync(0xffffffffu, ek);
+            if (ek >= 0 && lane == __ffs(same) - 1) atomicAdd(&hist[ek], __popc(same));
           }
         }
       }
@@ -495,9 +493,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int e = 0; e < E; ++e) lrow[e] = 0.f;
       if (valid) {
         if (p.K <= 8) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            if (k < p.K) lrow[se[k]] = sw[k];
+          for (int k = 0; k < p.K; ++k) {
+            const int e = sel_e[k * BM + row];
+            if (!(e & kDroppedBit)) lrow[e] = sel_p[k * BM + row];
+          }
         } else {
           for (int k = 0; k < p.K; ++k) {
             const size_t o = static_cast<size_t>(t) * p.K + k;
