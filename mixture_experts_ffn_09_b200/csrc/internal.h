@@ -63,6 +63,7 @@ cudaError_t launch_permute_scan(const int* blockcounts, int B, int E, int* block
 // slot, pos[slot] = row; block 0 also writes offsets (E + 1).
 // Slots whose in-block rank reaches the (clamped) block count, and slots
 // with the sentinel expert, get no row: pos = -1, slot_kept = 0.
+// blockbase / totals null: the kernel scans the block counts itself.
 cudaError_t launch_permute_scatter(const int* idx32, const int* blockbase, const int* totals,
                                    const int* blockcounts, int T, int K, int E, int* offsets,
                                    int* perm, int* pos, uint8_t* slot_kept, cudaStream_t s);

@@ -29,7 +29,10 @@ thread_local std::string g_last_error;
 std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
 std::atomic<int> g_fused_gather{0};
 std::atomic<int> g_pdl{0};   // programmatic dependent launch: opt-in
-std::atomic<int> g_debug_sync_ms{0};   // > 0: bounded wait after every kernel of a forward
+std::atomic<int> g_debug_sync_ms{0};
+// Block-count tables up to this many entries (blocks x experts) are scanned
+// inside the scatter kernel: each of its blocks reads the whole table.
+constexpr long long kScatterScansItself = 4096;   // > 0: bounded wait after every kernel of a forward
 
 // The tensor-core GEMM for one launch: CTA pairs pay off when experts have
 // enough rows to fill 256-row tiles.  With gather_perm the A rows are read
@@ -489,11 +492,15 @@ moe_status_t moe_ffn_forward_ex(const void* x, const void* router, const void* g
       if (r != cudaSuccess) return r;
       if (!debug_wait(dev, s, "capacity clamp")) return cudaErrorTimeout;
     }
-    r = moe::launch_permute_scan(bcount, L.B, E, bbase, totals, s);
-    if (r != cudaSuccess) return r;
-    if (!debug_wait(dev, s, "permute scan")) return cudaErrorTimeout;
-    r = moe::launch_permute_scatter(idx32, bbase, totals, bcount, Ti, K, E, offsets, perm, pos,
-                                    slot_kept, s);
+    // a small block-count table is scanned by the scatter blocks themselves
+    const bool own_scan = static_cast<long long>(L.B) * E <= kScatterScansItself;
+    if (!own_scan) {
+      r = moe::launch_permute_scan(bcount, L.B, E, bbase, totals, s);
+      if (r != cudaSuccess) return r;
+      if (!debug_wait(dev, s, "permute scan")) return cudaErrorTimeout;
+    }
+    r = moe::launch_permute_scatter(idx32, own_scan ? nullptr : bbase, own_scan ? nullptr : totals,
+                                    bcount, Ti, K, E, offsets, perm, pos, slot_kept, s);
     if (r != cudaSuccess) return r;
     if (!debug_wait(dev, s, "permute scatter")) return cudaErrorTimeout;
     if (fused_gather) return r;

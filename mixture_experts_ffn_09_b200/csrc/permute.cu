@@ -7,7 +7,8 @@
 // the result is deterministic and independent of scheduling.  Three kernels:
 //   scan    - one CTA per expert scans that expert's column of the router's
 //             32-token histograms: each block's first row within the expert
-//             and the expert's total;
+//             and the expert's total (for a small table the scatter blocks
+//             scan it themselves and this kernel does not run);
 //   scatter - one CTA per 32-token block ranks its slots within their
 //             expert (warp match + per-warp counts) and writes perm / pos;
 //             slots the router dropped, or past a capacity, get no row;
@@ -81,11 +82,35 @@ __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
+  if (!blockbase) {
+    // no scan kernel ran (small block-count table): each block scans the
+    // expert columns itself - the expert totals and the rows of each expert
+    // in earlier blocks, both in block order
+    // one warp per expert, lanes striding over the blocks
+    for (int e = warp; e < E; e += kScatterWarps) {
+      int before = 0, total = 0;
+      for (int b2 = lane; b2 < static_cast<int>(gridDim.x); b2 += 32) {
+        const int c = blockcounts[static_cast<size_t>(b2) * E + e];
+        before += b2 < b ? c : 0;
+        total += c;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        before += __shfl_xor_sync(0xffffffffu, before, o);
+        total += __shfl_xor_sync(0xffffffffu, total, o);
+      }
+      if (lane == 0) {
+        base[e] = before;
+        run[e] = total;                    // borrowed until the offsets exist
+      }
+    }
+    __syncthreads();
+  }
   if (threadIdx.x == 0) {
     int acc = 0;
     for (int e = 0; e < E; ++e) {
       off[e] = acc;
-      acc += totals[e];
+      acc += blockbase ? totals[e] : run[e];
     }
     off[E] = acc;
   }
@@ -93,7 +118,7 @@ __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
   if (b == 0)
     for (int e = threadIdx.x; e <= E; e += kScatterThreads) offsets[e] = off[e];
   for (int e = threadIdx.x; e < E; e += kScatterThreads) {
-    base[e] = off[e] + blockbase[static_cast<size_t>(b) * E + e];
+    base[e] = off[e] + (blockbase ? blockbase[static_cast<size_t>(b) * E + e] : base[e]);
     kept[e] = blockcounts[static_cast<size_t>(b) * E + e];
     run[e] = 0;
 #pragma unroll
