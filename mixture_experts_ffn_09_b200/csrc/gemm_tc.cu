@@ -429,7 +429,8 @@ cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params&
 }  // namespace
 
 cudaError_t launch_gemm_tc(int act, const void* A, int a_rows, const void* W, const int* offsets,
-                           int E, int T, int Kdim, int N, int w_rows_per_expert, const float* bias,
+                           int E, long long rows, int Kdim, int N, int w_rows_per_expert,
+                           const float* bias,
                            void* C, unsigned int* err, cudaStream_t s, const int* gather_perm,
                            int gather_K, int gather_rows) {
   CUtensorMap ma, mb;
@@ -451,11 +452,19 @@ cudaError_t launch_gemm_tc(int act, const void* A, int a_rows, const void* W, co
   p.bias = bias;
   p.err = err;
   const int bn_out = (act == kSiluGated) ? 128 : 256;
+  const long long n_tiles = (N + bn_out - 1) / bn_out;
   // upper bound on the tile count: every expert may add one partial row block
-  (void)T;
-  const long long tiles_bound =
-      (static_cast<long long>(a_rows) / BM + E) * ((N + bn_out - 1) / bn_out);
-  const int grid = static_cast<int>(tiles_bound < num_sms() ? tiles_bound : num_sms());
+  const long long tiles_bound = (static_cast<long long>(a_rows) / BM + E) * n_tiles;
+  // With at most 128 rows per expert on average (weight streaming) each
+  // touched expert has one row block and, rows >= E, all experts are
+  // likely touched: size the grid so that every CTA takes the same number of
+  // tiles.  A last wave of a few CTAs would stream its weight tiles at
+  // single-SM bandwidth while the rest of HBM sits idle.
+  long long tiles = tiles_bound;
+  if (rows <= 128LL * E) tiles = (rows < E ? rows : E) * n_tiles;
+  const long long sms = num_sms();
+  const long long waves = (tiles + sms - 1) / sms;
+  const int grid = static_cast<int>(waves > 0 ? (tiles + waves - 1) / waves : 1);
   if (gather) {
     if (act == kSiluGated) return launch_epi<kSiluGated, true>(ma, mb, p, grid, s);
     if (act == kReluBias) return launch_epi<kReluBias, true>(ma, mb, p, grid, s);

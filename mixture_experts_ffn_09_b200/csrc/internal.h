@@ -92,8 +92,9 @@ cudaError_t launch_gemm_simt_f32(int act, const float* A, const float* W, const 
 // With gather_perm set, A is x itself (gather_rows = T rows) and each tile's
 // rows are fetched by token index perm[row] / gather_K (TMA tile::gather4),
 // so the expert-sorted copy of x is never written.
+// rows = routed rows T*K (sizes the persistent grid).
 cudaError_t launch_gemm_tc(int act, const void* A, int a_rows, const void* W, const int* offsets,
-                           int E, int T, int Kdim, int N, int w_rows_per_expert,
+                           int E, long long rows, int Kdim, int N, int w_rows_per_expert,
                            const float* bias, void* C, unsigned int* err, cudaStream_t s,
                            const int* gather_perm = nullptr, int gather_K = 0,
                            int gather_rows = 0);

@@ -29,10 +29,10 @@ thread_local std::string g_last_error;
 std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
 std::atomic<int> g_fused_gather{0};
 std::atomic<int> g_pdl{0};   // programmatic dependent launch: opt-in
-std::atomic<int> g_debug_sync_ms{0};
+std::atomic<int> g_debug_sync_ms{0};   // > 0: bounded wait after every kernel of a forward
 // Block-count tables up to this many entries (blocks x experts) are scanned
 // inside the scatter kernel: each of its blocks reads the whole table.
-constexpr long long kScatterScansItself = 4096;   // > 0: bounded wait after every kernel of a forward
+constexpr long long kScatterScansItself = 4096;
 
 // The tensor-core GEMM for one launch: CTA pairs pay off when experts have
 // enough rows to fill 256-row tiles.  With gather_perm the A rows are read
@@ -47,8 +47,8 @@ cudaError_t launch_gemm_bf16(int act, const void* A, int a_rows, const void* W,
   if (pair)
     return moe::launch_gemm_tc_pair(act, A, a_rows, W, offsets, E, Kdim, N, w_rows, bias, C, err, s,
                                     gather_perm, K, T);
-  return moe::launch_gemm_tc(act, A, a_rows, W, offsets, E, T, Kdim, N, w_rows, bias, C, err, s,
-                             gather_perm, K, T);
+  return moe::launch_gemm_tc(act, A, a_rows, W, offsets, E, static_cast<long long>(T) * K, Kdim, N,
+                             w_rows, bias, C, err, s, gather_perm, K, T);
 }
 
 __device__ unsigned int g_device_error;   // per device: bounded waits that gave up
