@@ -184,10 +184,14 @@ def oracle_rate(w, d, budget_s: float, first_n: int = 8):
                           d["b1"], d["b2"])
         return time.perf_counter() - t0
 
+    # a call has a large fixed cost (it streams every expert's float64
+    # weights), so the sample grows until one call takes about the budget
     n = min(first_n, w.T)
     t = run(n)
-    if t < budget_s / 3 and n < w.T:
-        n = int(min(w.T, max(n + 1, n * (budget_s / max(t, 1e-6)))))
+    for _ in range(4):
+        if t >= budget_s / 2 or n >= w.T:
+            break
+        n = int(min(w.T, max(2 * n, n * (budget_s / max(t, 1e-6)))))
         t = run(n)
     return n / t, n, t
 
