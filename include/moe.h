@@ -322,6 +322,11 @@ MOE_API moe_status_t moe_device_status(void* stream);
  */
 MOE_API moe_status_t moe_device_error_peek(unsigned int* word);
 
+/* Number of kernels this library has launched in the process so far (all
+   devices, all entry points; launches the CUDA runtime accepted).  A forward
+   launches 6 to 9 kernels depending on its size and options. */
+MOE_API unsigned long long moe_kernel_launches(void);
+
 /* Comma-separated names of the sites set in an error word (static storage
    of the calling thread, overwritten by the next call). */
 MOE_API const char* moe_error_sites(unsigned int word);

@@ -13,8 +13,11 @@
 namespace moe {
 
 // Programmatic dependent launch between the kernels of a forward (process
-// wide, on by default; see moe_set_pdl).
+// wide, off by default; see moe_set_pdl).
 bool pdl_enabled();
+
+// Counts a kernel launch that was accepted (moe_kernel_launches).
+void note_launch();
 
 // Error bits a kernel ORs into the per-device error word.  A timed-out
 // wait also sets the bit of its site (kernel and role), so the host can say
@@ -97,7 +100,9 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e == cudaSuccess) note_launch();
+  return e;
 }
 
 // ------------------------------------------------------------- mbarrier

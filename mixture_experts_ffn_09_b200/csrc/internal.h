@@ -107,6 +107,7 @@ cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* 
                                 int gather_rows = 0);
 
 int num_sms();
+unsigned long long kernel_launches();   // accepted launches so far (note_launch)
 
 // One CTA waiting (bounded) on an mbarrier nothing arrives at.
 cudaError_t launch_bounded_wait_probe(unsigned long long timeout_ns, unsigned int* err,

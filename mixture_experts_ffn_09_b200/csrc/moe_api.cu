@@ -586,6 +586,8 @@ moe_status_t moe_device_error_peek(unsigned int* word) {
   return MOE_OK;
 }
 
+unsigned long long moe_kernel_launches(void) { return moe::kernel_launches(); }
+
 int moe_set_debug_sync(int timeout_ms) { return g_debug_sync_ms.exchange(timeout_ms > 0 ? timeout_ms : 0); }
 
 moe_status_t moe_device_status(void* stream) {
@@ -637,6 +639,10 @@ int moe_profile_read(float* ms, int n_stages) {
 
 namespace moe {
 bool pdl_enabled() { return g_pdl.load() != 0; }
+
+std::atomic<unsigned long long> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+unsigned long long kernel_launches() { return g_launches.load(); }
 
 int num_sms() {
   int dev = 0;

@@ -118,7 +118,9 @@ __global__ void bounded_wait_probe_kernel(unsigned long long timeout_ns, unsigne
 cudaError_t launch_bounded_wait_probe(unsigned long long timeout_ns, unsigned int* err,
                                       cudaStream_t s) {
   bounded_wait_probe_kernel<<<1, 32, 0, s>>>(timeout_ns, err);
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) note_launch();
+  return e;
 }
 
 cudaError_t launch_capacity_clamp(int* blockcounts, int B, int E, int T, int K, int seq_len,

@@ -105,6 +105,8 @@ def lib() -> ctypes.CDLL:
         L.moe_device_status.restype = i32
         L.moe_device_error_peek.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         L.moe_device_error_peek.restype = i32
+        L.moe_kernel_launches.argtypes = []
+        L.moe_kernel_launches.restype = ctypes.c_ulonglong
         L.moe_error_sites.argtypes = [ctypes.c_uint]
         L.moe_error_sites.restype = ctypes.c_char_p
         L.moe_profile_enable.argtypes = [i32]
@@ -409,6 +411,11 @@ def device_error_peek() -> int:
     w = ctypes.c_uint(0)
     _check(lib().moe_device_error_peek(ctypes.byref(w)))
     return int(w.value)
+
+
+def kernel_launches() -> int:
+    """Kernels this library has launched in the process so far."""
+    return int(lib().moe_kernel_launches())
 
 
 def error_sites(word: int) -> str:

@@ -422,3 +422,32 @@ def test_forward_replays_from_a_cuda_graph(gemm_mode):
         torch.cuda.synchronize()
         assert torch.equal(out, ref[0]) and torch.equal(sel, ref[1]) and torch.equal(w, ref[2])
     assert moe.device_status() == moe.MOE_OK
+
+
+def test_kernel_launch_count_per_forward():
+    """A forward launches router, scatter, gather, gate_up, down and combine;
+    the scan kernel only runs for block-count tables of more than 4096
+    entries, and the capacity clamp and the balance finaliser add one each."""
+    import torch
+    from mixture_experts_ffn_09_b200 import moe
+
+    def launches(T, E, **opts):
+        d = synth.random_case(23, T, 64, 64, E, dtype="bf16", weight_std=0.05)
+        dev = PL.to_device(d)
+        x = dev["x"]
+        ws = torch.empty(moe.workspace_size(T, 64, 64, E, 2, moe.BF16), dtype=torch.uint8,
+                         device="cuda")
+        out = torch.empty_like(x)
+        sel = torch.empty(T, 2, dtype=torch.int64, device="cuda")
+        w = torch.empty(T, 2, dtype=torch.float32, device="cuda")
+        n0 = moe.kernel_launches()
+        moe.ffn_forward_ex(x, dev["router"], dev["gate_up_proj"], dev["down_proj"], E, 2, True,
+                           moe.ACT_SILU_GATED, out, sel, w, None, None, None, None, ws, **opts)
+        n = moe.kernel_launches() - n0
+        assert moe.device_status() == moe.MOE_OK
+        return n
+
+    assert launches(256, 8) == 6                     # 8 blocks x 8 experts: scanned in scatter
+    assert launches(4096, 64) == 7                   # 128 x 64 entries: the scan kernel runs
+    bal = torch.empty(4, dtype=torch.float32, device="cuda")
+    assert launches(256, 8, capacity_factor=1.0, balance=bal) == 8
