@@ -158,7 +158,8 @@ __global__ void __launch_bounds__(kWarps * 32) router_topk_kernel(RouteArgs a) {
       key[i] = -INFINITY;
       if (e < E) {
         sc[i] = a.score == 0 ? expf(l[i] - m) / s : 1.f / (1.f + expf(-l[i]));
-        key[i] = a.sel_bias ? sc[i] + __ldg(a.sel_bias + e) : l[i];
+        const float kb = a.sel_bias ? sc[i] + __ldg(a.sel_bias + e) : l[i];
+        key[i] = isnan(kb) ? -INFINITY : kb;   // NaN never ranks: keep every key orderable
         if (a.bal_partial) bal[e] += sc[i];
       }
     }

@@ -270,8 +270,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     // sum the split partials in rank order, add the bias, write the logits
     float lmax = -INFINITY;
     for (int e = e_lo; e < e_hi; ++e) {
-      float v = lrow[e];
-      for (int q = 1; q < p.S; ++q) v += part[(q * BM + row) * C::PART_STRIDE + e];
+      // padding rows were not copied: they reduce to zeros (their results
+      // are never stored, but must stay well defined)
+      float v = valid ? lrow[e] : 0.f;
+      for (int q = 1; q < p.S; ++q)
+        if (valid) v += part[(q * BM + row) * C::PART_STRIDE + e];
       if (p.bias) v += __ldg(p.bias + e);
       if (valid && p.logits) p.logits[static_cast<size_t>(t) * E + e] = v;
       if (isnan(v)) v = -INFINITY;
@@ -294,12 +297,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     // score of expert e: softmax probability or sigmoid of the logit
     auto score = [&](int e) {
-      const float l = lrow[e];
+      const float l = e < E ? lrow[e] : -INFINITY;
       return p.score == 0 ? expf(l - m) / s : 1.f / (1.f + expf(-l));
     };
     // ranking key: the logit (monotone in either score) unless a selection
-    // bias is added to the score
-    auto key = [&](int e) { return p.sel_bias ? score(e) + __ldg(p.sel_bias + e) : lrow[e]; };
+    // bias is added to the score; a NaN key (from NaN inputs) ranks as -inf,
+    // so every expert stays orderable and a choice is always a real expert
+    auto key = [&](int e) {
+      const float k = p.sel_bias ? score(e) + __ldg(p.sel_bias + e) : lrow[e];
+      return isnan(k) ? -INFINITY : k;
+    };
     if (p.K <= 8) {
       // each slice keeps a sorted list of its best entries (value
       // descending, index ascending: a later equal value never overtakes, so

@@ -178,3 +178,28 @@ def test_route_ex_entry_point():
     np.testing.assert_array_equal(sel.cpu().numpy()[clear], r["selected_experts"][clear])
     np.testing.assert_allclose(wt.cpu().numpy()[clear], r["routing_weights"][clear], atol=1e-5)
     np.testing.assert_array_equal(kept.cpu().numpy().astype(bool)[clear], r["active"][clear])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("score", ["softmax", "sigmoid"])
+def test_nan_tokens_are_contained(dtype, score):
+    """Tokens whose x holds NaN still get K real experts (NaN scores rank
+    last), nothing faults, and every other token's result is bit for bit the
+    one it gets without the NaN tokens present (rows are independent)."""
+    import torch
+    d = synth.random_case(301, 200, 64, 96, 8, dtype=dtype, weight_std=0.1)
+    bias = np.random.default_rng(4).normal(0, 0.05, 8).astype(np.float32)
+    clean = PL.to_device(d)
+    dirty = dict(clean)
+    xd = clean["x"].clone()
+    bad = [0, 5, 77, 199]
+    xd[bad] = float("nan")
+    dirty["x"] = xd
+    opts = dict(score=score, selection_bias=bias)
+    a = run_gpu_ex(clean, 8, 3, True, "silu_gated", **dict(opts))
+    b = run_gpu_ex(dirty, 8, 3, True, "silu_gated", **dict(opts))
+    assert ((b["sel"] >= 0) & (b["sel"] < 8)).all()
+    keep = np.setdiff1d(np.arange(200), bad)
+    np.testing.assert_array_equal(b["sel"][keep], a["sel"][keep])
+    np.testing.assert_array_equal(b["w"][keep], a["w"][keep])
+    np.testing.assert_array_equal(b["out"][keep], a["out"][keep])
