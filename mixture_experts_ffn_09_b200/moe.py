@@ -383,7 +383,7 @@ def set_gemm_mode(mode: int) -> int:
 
 def set_pdl(on: bool) -> bool:
     """Programmatic dependent launch between a forward's kernels (default
-    on); returns the previous setting."""
+    off; see moe_set_pdl in include/moe.h); returns the previous setting."""
     return bool(lib().moe_set_pdl(int(bool(on))))
 
 
