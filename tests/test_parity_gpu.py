@@ -133,6 +133,9 @@ CASES = [
     (77, 50, 30, 4, 2, "relu", "f32"),
     (1, 8, 8, 1, 1, "silu_gated", "f32"),           # one token, one expert
     (129, 264, 520, 1, 1, "silu_gated", "bf16"),    # one expert: a plain FFN
+    (160, 128, 128, 16, 12, "silu_gated", "bf16"),  # K > 8: the router's round-per-choice path
+    (150, 96, 64, 100, 6, "silu_gated", "bf16"),    # E in (64, 128]: 128-column router tile
+    (60, 32, 32, 20, 10, "silu_gated", "f32"),      # K > 8 on the fp32 router
 ]
 
 

@@ -143,6 +143,16 @@ def test_all_extensions_together():
               L=64)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_all_extensions_with_more_than_eight_choices(dtype):
+    """K > 8 takes the routers' round-per-choice path: every extension at
+    once there too."""
+    d = synth.random_case(52, 256, 64, 64, 16, dtype=dtype, weight_std=0.3 if dtype == "f32" else 0.05)
+    bias = np.random.default_rng(5).normal(0, 0.03, 16).astype(np.float32)
+    check_ext(d, 16, 10, True, "silu_gated", dtype, score="sigmoid", sel_bias=bias, th=0.05,
+              cf=1.0, L=64)
+
+
 def test_relu_expert_with_capacity_and_threshold():
     d = synth.random_case(61, 200, 72, 80, 5, act="relu", dtype="bf16", weight_std=0.1)
     check_ext(d, 5, 3, True, "relu", "bf16", th=0.25, cf=1.0, L=32)
