@@ -508,7 +508,7 @@ def run_ours(args, w):
         "metric": METRIC, "value": round(tokens_per_s, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
-        "data": "synthetic (seeded, shapes of the pages' workloads; random-init weights)",
+        "data": "synthetic (seeded, shapes of the published workloads; random-init weights)",
         "config": dict(workload_config(w, world), gemm=args.gemm, pdl=args.pdl,
                        **({"routing": {"score": args.score, "selection_bias_std": args.selection_bias,
                                        "dynamic_threshold": args.dynamic_threshold,
@@ -590,7 +590,7 @@ def run_reference(args, w):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(secs / max(args.steps, 1) * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded, shapes of the pages' workloads; random-init weights)",
+        "data": "synthetic (seeded, shapes of the published workloads; random-init weights)",
         "config": workload_config(w, 1), "impl": "reference",
         "cpu_baseline": {"value": round(rate, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},

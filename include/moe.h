@@ -218,8 +218,8 @@ MOE_API moe_status_t moe_route_ex(const void* x, const void* router, const float
  * memory at call time: code running where a device allocation is not
  * permitted or not available to it, such as a plugin or callback of another
  * runtime that owns all device memory and hands the plugin only its inputs
- * and outputs.  The pages have no counterpart; it is an addition of this
- * library.
+ * and outputs.  The cited descriptions of the layer have no counterpart;
+ * it is an addition of this library.
  *
  * Same arguments and results as moe_ffn_forward, without the workspace:
  * the scratch lives in one static device array of

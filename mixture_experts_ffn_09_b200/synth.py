@@ -5,7 +5,7 @@ layer's arithmetic (no routing, no softmax, no expert maths), so both the
 float64 oracle and the CUDA path can be fed from it without sharing any
 computation.
 
-Workloads follow the shapes of the pages' problems:
+Workloads follow the shapes of the published problems:
 
 * the Flax exercise "Mixture-of-Experts FFN" (crackedaicode.com, section
   "Problem"): Dense(F)->ReLU->Dense(D) experts with biases and a biased
@@ -15,7 +15,7 @@ Workloads follow the shapes of the pages' problems:
 * three bf16 layers of Mixtral-8x7B, fine-grained many-expert and decode
   shapes.
 
-Recipe (the one the design doc states):
+Recipe:
 
 * small float32 workloads draw from ONE ``numpy.random.default_rng(seed)``
   in the order x, router, [router_bias], gate_up_proj, down_proj, [b1, b2];

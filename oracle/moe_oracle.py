@@ -6,7 +6,7 @@ and the CPU-baseline leg of the benchmark script may use it.  It shares no
 code with the CUDA library (no kernels, headers, tables or helpers) and
 imports nothing from the product package.
 
-It is written to be read against the pages, not to be fast:
+It is written to be read against the sources it cites, not to be fast:
 
 * every expert is evaluated on every token and the selected outputs are then
   gathered, exactly as the Flax exercise "Mixture-of-Experts FFN"
@@ -19,7 +19,7 @@ It is written to be read against the pages, not to be fast:
   check the Dew "Mixture of experts" page describes under "Expert
   computation and placement" (float64 arithmetic on the rounded operands).
 
-Readings where the pages leave a step open (each is listed in the design doc):
+Readings taken where those sources leave a step open:
 
 * gate_up_proj rows [0, F) are the gate projection and rows [F, 2F) the up
   projection (the plain concatenation order of the name);
@@ -35,7 +35,7 @@ Readings where the pages leave a step open (each is listed in the design doc):
 
 Routing extensions ("Mixture of experts", dewml.dev, "Router behavior" and
 "Expert computation and placement"; ES-MoE API page, "ESMoE" settings and
-"Balancing objectives"), with the readings the design doc lists:
+"Balancing objectives"), with these readings:
 
 * sigmoid scores: each expert's score is sigmoid(logit) on its own;
 * a selection bias is added to the scores only to choose the experts; the
@@ -50,7 +50,7 @@ Routing extensions ("Mixture of experts", dewml.dev, "Router behavior" and
 
 Parity status: every function here is pinned by the CPU tests in
 ``tests/test_oracle_pins.py`` (worked example, closed forms, invariants,
-brute force, library special cases).  The pages' own seeded outputs (Flax
+brute force, library special cases).  The sources' own seeded outputs (Flax
 PRNG, mojolearn's generator) cannot be reproduced and are not claimed.
 """
 from __future__ import annotations

@@ -1,6 +1,6 @@
 """Pins of the oracle's routing extensions (CPU only): sigmoid scores, the
 selection-only bias, ES-MoE's dynamic threshold, the capacity factor and the
-balancing statistics - each tied to hand-worked cases from the pages'
+balancing statistics - each tied to hand-worked cases from the cited
 definitions, closed forms, or an independent formulation."""
 import itertools
 

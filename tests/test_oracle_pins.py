@@ -1,7 +1,7 @@
 """Pins of the float64 oracle to facts outside itself (CPU only).
 
-Each test ties one part of the oracle to something the pages or the
-mathematics fix: the exercise's worked example, the parameter-count closed
+Each test ties one part of the oracle to something the cited sources or
+the mathematics fix: the exercise's worked example, the parameter-count closed
 form, invariants of the weights, lower-index tie-breaking, token
 permutation equivariance, brute force on tiny inputs, and special cases that
 reduce to library routines (torch float64 linear algebra, the installed
