@@ -461,20 +461,44 @@ template <int EPI, bool GATHER>
 cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params& p, int clusters,
                        cudaStream_t s) {
   static std::mutex mu;
-  static bool done[64] = {};
+  static int resident[64] = {};    // pairs that fit on the device at once (0: not asked yet)
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
+  int fit = 0;
   {
     std::lock_guard<std::mutex> lock(mu);
-    if (dev < 0 || dev >= 64 || !done[dev]) {
+    if (dev < 0 || dev >= 64 || resident[dev] == 0) {
       err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<EPI, GATHER>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kSmemBytes));
       if (err != cudaSuccess) return err;
-      if (dev >= 0 && dev < 64) done[dev] = true;
+      // the grid is persistent: every pair should be resident from the start
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * clusters);
+      cfg.blockDim = dim3(THREADS);
+      cfg.dynamicSmemBytes = kSmemBytes;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 2;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<EPI, GATHER>, &cfg) !=
+              cudaSuccess ||
+          n <= 0) {
+        cudaGetLastError();            // the query is advisory: fall back to one pair per 2 SMs
+        n = num_sms() / 2;
+      }
+      fit = n;
+      if (dev >= 0 && dev < 64) resident[dev] = n;
+    } else {
+      fit = resident[dev];
     }
   }
+  if (clusters > fit) clusters = fit;
   return launch_k(grouped_gemm_pair_kernel<EPI, GATHER>, dim3(2 * clusters), dim3(THREADS),
                   kSmemBytes, s, pdl_enabled(), 2, a, b, p);
 }
