@@ -454,3 +454,35 @@ def test_kernel_launch_count_per_forward():
     assert launches(4096, 64) == 7                   # 128 x 64 entries: the scan kernel runs
     bal = torch.empty(4, dtype=torch.float32, device="cuda")
     assert launches(256, 8, capacity_factor=1.0, balance=bal) == 8
+
+
+def _random_shapes(n, seed):
+    """Seeded layer shapes across the supported ranges: bf16 needs D and F
+    multiples of 8, any sizes on float32."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        dtype = "bf16" if i % 3 else "f32"
+        step = 8 if dtype == "bf16" else 1
+        T = int(rng.integers(1, 700))
+        D = int(rng.integers(1, 64)) * step
+        F = int(rng.integers(1, 64)) * step
+        E = int(rng.integers(1, 80))
+        K = int(rng.integers(1, min(E, 10) + 1))
+        act = "relu" if rng.random() < 0.3 else "silu_gated"
+        out.append((T, D, F, E, K, act, dtype, int(rng.integers(1, 3))))
+    return out
+
+
+@pytest.mark.parametrize("T,D,F,E,K,act,dtype,mode", _random_shapes(12, 2026))
+def test_random_shapes_sweep(T, D, F, E, K, act, dtype, mode):
+    """Seeded random layers (token count, widths, expert count, top-k,
+    activation, dtype, GEMM variant): every token against the oracle."""
+    from mixture_experts_ffn_09_b200 import moe
+    prev = moe.set_gemm_mode(mode)
+    try:
+        d = synth.random_case(3000 + T + E, T, D, F, E, act=act, dtype=dtype,
+                              weight_std=0.3 if dtype == "f32" else 0.05)
+        _full_check(d, E, K, True, act, dtype)
+    finally:
+        moe.set_gemm_mode(prev)
