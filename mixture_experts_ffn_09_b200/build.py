@@ -10,6 +10,7 @@ inspected; calls that reach the device then fail with a CUDA error).
 from __future__ import annotations
 
 import argparse
+import fcntl
 import glob
 import os
 import shutil
@@ -53,9 +54,23 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile and link when a source is newer than the library (or on
+    force).  Processes that call this at once (one per GPU) serialise on a
+    lock file; those that waited find the library current and return."""
     if not force and up_to_date():
         return LIB
     os.makedirs(OBJ, exist_ok=True)
+    with open(os.path.join(OBJ, ".lock"), "w") as lk:
+        fcntl.flock(lk, fcntl.LOCK_EX)
+        try:
+            if not force and up_to_date():
+                return LIB
+            return _build_locked(verbose)
+        finally:
+            fcntl.flock(lk, fcntl.LOCK_UN)
+
+
+def _build_locked(verbose: bool) -> str:
     cc = nvcc()
     extra = ["-Xptxas", "-v"] if verbose else []
 
@@ -71,7 +86,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
     with ThreadPoolExecutor(max(1, min(8, os.cpu_count() or 1))) as ex:
         objs = list(ex.map(compile_one, _sources()))
-    tmp = LIB + ".tmp"
+    tmp = f"{LIB}.{os.getpid()}.tmp"
     cmd = [cc, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs, "-cudart", "static"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
