@@ -319,6 +319,10 @@ def run_ours(args, w):
     build.build()
     moe.set_gemm_mode({"auto": moe.GEMM_AUTO, "1sm": moe.GEMM_1SM, "2sm": moe.GEMM_2SM}[args.gemm])
     moe.set_pdl(args.pdl)
+    if args.tail_swap is not None:
+        moe.set_tail_swap(args.tail_swap)
+    tail_swap = moe.set_tail_swap(0)
+    moe.set_tail_swap(tail_swap)
     if args.debug_sync_ms > 0:
         moe.set_debug_sync(args.debug_sync_ms)
     dev = torch.device("cuda", local)
@@ -509,7 +513,7 @@ def run_ours(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded, shapes of the published workloads; random-init weights)",
-        "config": dict(workload_config(w, world), gemm=args.gemm, pdl=args.pdl,
+        "config": dict(workload_config(w, world), gemm=args.gemm, pdl=args.pdl, tail_swap=tail_swap,
                        **({"routing": {"score": args.score, "selection_bias_std": args.selection_bias,
                                        "dynamic_threshold": args.dynamic_threshold,
                                        "capacity_factor": args.capacity_factor,
@@ -619,6 +623,9 @@ def main(argv=None):
     ap.add_argument("--capacity-factor", type=float, default=0.0)
     ap.add_argument("--seq-len", type=int, default=0)
     ap.add_argument("--balance", action="store_true", help="also compute the balancing statistics")
+    ap.add_argument("--tail-swap", type=int, default=None,
+                    help="rows up to which an expert's last CTA-pair tile runs with swapped "
+                         "operands (0..255, 0 = off; default: the library's)")
     ap.add_argument("--pdl", action="store_true",
                     help="launch the kernels with programmatic dependent launch (off by default)")
     ap.add_argument("--watchdog", type=float, default=120.0,

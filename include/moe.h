@@ -262,6 +262,21 @@ MOE_API moe_status_t moe_ffn_forward_noalloc(const void* x, const void* router,
 MOE_API int moe_set_gemm_mode(int mode);
 
 /*
+ * Short expert tails on the CTA-pair GEMM (process-wide setting).  An
+ * expert's routed rows fill 256-row tiles; when its last tile holds at most
+ * max_rows rows, that tile runs with the operands swapped: 256 weight rows
+ * as the MMA's M and the tail's rows (rounded up to 16, 32, 64 or 128) as
+ * its N, instead of a full 256-row tile that is mostly padding.  max_rows in
+ * 0..MOE_TAIL_SWAP_MAX; 0 turns it off.  The SiLU-gated GEMM swaps only when
+ * F is a multiple of 16.  Results agree with the unswapped tile up to fp32
+ * summation order.  Returns the previous setting, or -1 if max_rows is out
+ * of range (nothing changes).
+ */
+#define MOE_TAIL_SWAP_DEFAULT 128
+#define MOE_TAIL_SWAP_MAX 128
+MOE_API int moe_set_tail_swap(int max_rows);
+
+/*
  * Whether the bf16 gate_up GEMM fetches its token rows from x by index
  * (TMA tile::gather4, four rows per copy) instead of from an expert-sorted
  * copy written by a separate gather kernel.  Results are bit-identical.

@@ -29,7 +29,19 @@
 // [128,256) up in both CTAs, exactly as in the one-CTA kernel.
 //
 // A pair tile covers 256 rows of one expert; rows past the expert's end are
-// computed and not stored.  No load uses cluster multicast.
+// computed and not stored.  The exception is an expert's last row block when
+// it holds at most `swap_max` rows (a short tail): that tile runs with the
+// operands swapped.  The weight rows become the MMA's M = 256 and the tail's
+// token rows its N (rounded up to 16, half from each CTA), so the tensor
+// cores do not spend a full 256-row tile on a few rows.  For the gated
+// expert each CTA stages its 64 gate rows and the matching 64 up rows
+// interleaved in groups of 16, so the gate and up values of one feature land
+// in TMEM lanes i and i^16 of the same warp and meet through one shuffle.
+// The epilogue writes the transposed result straight to the row-major output.
+// A swapped k-block takes two copies per CTA, as a regular one does: the
+// token rows in one box of 8, 16, 32 or 64 rows (N = 16..128), and the
+// interleaved gate/up rows through one 4-D view of the weights.
+// No load uses cluster multicast.
 #include <mutex>
 
 #include "common.cuh"
@@ -48,6 +60,13 @@ constexpr int B_BYTES = (BN_MMA / 2) * BK * 2;  // 16 KB (this CTA's half)
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
+constexpr int WB_BOX = 16;      // gate (then up) rows per group of the interleaved staging
+constexpr int kSwapMax = 128;   // longest tail that may run swapped (N = 128)
+
+// Token-row views for swapped tails: box heights 8, 16, 32 and 64 rows.
+struct TokMaps {
+  CUtensorMap m[4];
+};
 
 enum { kSiluGated = 0, kReluBias = 1, kBias = 2 };
 
@@ -63,6 +82,7 @@ struct Params {
   __nv_bfloat16* out;
   const float* bias;
   unsigned int* err;
+  int swap_max;       // an expert's last block of at most this many rows runs swapped (0: never)
 };
 
 struct Tail {
@@ -105,6 +125,15 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d_pair(const CUtensorMap* map, uint32_t bar_cluster_addr,
+                                                 void* dst, int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(c1), "r"(c2),
+      "r"(c3)
       : "memory");
 }
 // Gathered variant: 4 token rows of x (box 64 x 1) into 512 bytes of this
@@ -164,6 +193,18 @@ __device__ __forceinline__ void decode_tile(const Tail* st, int E, int n_tiles, 
   m_blk = local - n_blk * mt;
 }
 
+// Rows of a swapped tail tile (1..255), or 0 for a regular tile.  Every row
+// block but an expert's last has more than 255 rows left, so only the last
+// can qualify.
+__device__ __forceinline__ int swap_rows(const Tail* st, int swap_max, int e, int m_blk) {
+  const int left = st->off[e + 1] - st->off[e] - m_blk * BMP;
+  return left <= swap_max ? left : 0;
+}
+// The swapped tile's N: 16, 32, 64 or 128 (index 0..3 of the token views).
+__device__ __forceinline__ int swap_idx(int rows) {
+  return rows <= 16 ? 0 : rows <= 32 ? 1 : rows <= 64 ? 2 : 3;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -185,7 +226,9 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* rowp, int col0, int n
 template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
-                             const __grid_constant__ CUtensorMap tmB, const Params p) {
+                             const __grid_constant__ CUtensorMap tmB,
+                             const __grid_constant__ CUtensorMap tmGU,
+                             const __grid_constant__ TokMaps tmT, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   if ((smem_u32(smem_raw) & 1023u) != 0) {   // the ring needs 1024-byte alignment
@@ -221,6 +264,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (!GATHER && p.swap_max > 0) {
+      for (int j = 0; j < 4; ++j) tma_prefetch_desc(&tmT.m[j]);
+      if (EPI == kSiluGated) tma_prefetch_desc(&tmGU);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(&st->tmem_base, TMEM_COLS);
@@ -276,6 +323,40 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       bool ok = true;
+      const int sw = GATHER ? 0 : swap_rows(st, p.swap_max, e, m_blk);
+      if (sw) {
+        // swapped tail: this CTA's weight rows into the B slot, its half of
+        // the tail's token rows (nt/2) into the A slot
+        const int si = swap_idx(sw);
+        const int nt = 16 << si;
+        const int row_tok = st->off[e] + m_blk * BMP + static_cast<int>(rank) * (nt / 2);
+        // gated: the first 16-row group of this CTA's 64 features, counted in
+        // the weights' 16-row groups (the gated swap requires F % 16 == 0)
+        const int g0 = (e * p.b_rows + n_blk * 128 + static_cast<int>(rank) * 64) / WB_BOX;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          int good = 1;
+          if (lane == 0) {
+            good = mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err, SITE_PAIR_PRODUCER) ? 1 : 0;
+            if (good && leader) mbar_arrive_expect_tx(&st->full[stage], 2 * B_BYTES + nt * BK * 2);
+          }
+          if (!__shfl_sync(0xffffffffu, good, 0)) { ok = false; break; }
+          const uint32_t fb = map_to_rank(&st->full[stage], 0);
+          if (lane == 0) {
+            // box (64 k, 16 rows, gate/up, 4 groups) lands as smem rows
+            // 32q + i (gate) and 32q + 16 + i (up) of group q
+            if (EPI == kSiluGated)
+              tma_load_4d_pair(&tmGU, fb, sB + stage * B_BYTES, kb * BK, 0, 0, g0);
+            else
+              tma_load_2d_pair(&tmB, fb, sB + stage * B_BYTES, kb * BK, rowB);
+            tma_load_2d_pair(&tmT.m[si], fb, sA + stage * A_BYTES, kb * BK, row_tok);
+            used |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        continue;
+      }
       for (int kb = 0; kb < p.num_kb; ++kb) {
         int good = 1;
         if (lane == 0) {
@@ -323,17 +404,40 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const uint32_t d = tmem + acc * BN_MMA;
         bool ok = true;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&st->full[stage], phase, abort, p.err, SITE_PAIR_MMA)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
-          const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+        int sw = 0;
+        if (!GATHER && p.swap_max > 0) {
+          int e, m_blk, n_blk;
+          decode_tile(st, E, n_tiles, t, e, m_blk, n_blk);
+          sw = swap_rows(st, p.swap_max, e, m_blk);
+        }
+        if (sw) {
+          // swapped tail: A = the weight rows (B slot), B = the token rows (A slot)
+          const uint32_t idesc_sw = idesc_bf16_f32(BMP, 16 << swap_idx(sw));
+          for (int kb = 0; kb < p.num_kb; ++kb) {
+            if (!mbar_wait(&st->full[stage], phase, abort, p.err, SITE_PAIR_MMA)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t w0 = smem_u32(sB + stage * B_BYTES);
+            const uint32_t x0 = smem_u32(sA + stage * A_BYTES);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            umma_bf16_pair(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
-                           (kb | k) != 0 ? 1u : 0u);
-          umma_commit_pair(&st->empty[stage]);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            for (int k = 0; k < BK / 16; ++k)
+              umma_bf16_pair(d, sw128_kmajor_desc(w0 + k * 32), sw128_kmajor_desc(x0 + k * 32),
+                             idesc_sw, (kb | k) != 0 ? 1u : 0u);
+            umma_commit_pair(&st->empty[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          }
+        } else {
+          for (int kb = 0; kb < p.num_kb; ++kb) {
+            if (!mbar_wait(&st->full[stage], phase, abort, p.err, SITE_PAIR_MMA)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
+            const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)
+              umma_bf16_pair(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
+                             (kb | k) != 0 ? 1u : 0u);
+            umma_commit_pair(&st->empty[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          }
         }
         if (!ok) break;
         umma_commit_pair(&st->tfull[acc]);
@@ -357,10 +461,65 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool got = mbar_wait(&st->tfull[acc], aph, abort, p.err, SITE_PAIR_EPILOGUE);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
+      const uint32_t tb = tmem + (static_cast<uint32_t>(lane_base) << 16) + acc * BN_MMA;
+      const int sw = GATHER ? 0 : swap_rows(st, p.swap_max, e, m_blk);
+      if (sw) {
+        // swapped tail: this thread's TMEM lane is one weight row (an output
+        // feature), its columns the tail's token rows
+        const int row0 = st->off[e] + m_blk * BMP;
+        const int nchunks = (sw + 31) >> 5;
+        if (EPI == kSiluGated) {
+          // lane i < 16 holds gate, lane i + 16 up, of the same feature f
+          const bool hi = lane >= 16;
+          const int f = n_blk * 128 + static_cast<int>(rank) * 64 + (warp & 3) * WB_BOX + (lane & 15);
+          const bool fvalid = f < p.n_out;
+#pragma unroll 1
+          for (int c = 0; c < nchunks; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tb + c * 32, v);
+            tmem_ld_wait();
+            // the low lane finishes tokens 32c..32c+15, the high lane 32c+16..32c+31
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float give = __uint_as_float(hi ? v[j] : v[16 + j]);
+              const float got = __shfl_xor_sync(0xffffffffu, give, 16);
+              const float g = hi ? got : __uint_as_float(v[j]);
+              const float u = hi ? __uint_as_float(v[16 + j]) : got;
+              const int tok = c * 32 + (hi ? 16 : 0) + j;
+              if (fvalid && tok < sw)
+                p.out[static_cast<size_t>(row0 + tok) * p.n_out + f] =
+                    __float2bfloat16_rn(g / (1.f + __expf(-g)) * u);
+            }
+          }
+        } else {
+          const int dcol = n_blk * 256 + static_cast<int>(rank) * 128 + lane_base + lane;
+          const bool dvalid = dcol < p.n_out;
+          const float b =
+              (p.bias && dvalid) ? __ldg(p.bias + static_cast<size_t>(e) * p.n_out + dcol) : 0.f;
+#pragma unroll 1
+          for (int c = 0; c < nchunks; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tb + c * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int tok = c * 32 + j;
+              if (dvalid && tok < sw) {
+                float a = __uint_as_float(v[j]) + b;
+                if (EPI == kReluBias) a = fmaxf(a, 0.f);
+                p.out[static_cast<size_t>(row0 + tok) * p.n_out + dcol] = __float2bfloat16_rn(a);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+        continue;
+      }
       const int grow = st->off[e] + m_blk * BMP + static_cast<int>(rank) * BMC + lane_base + lane;
       const bool rvalid = grow < st->off[e + 1];
       __nv_bfloat16* rowp = p.out + static_cast<size_t>(rvalid ? grow : 0) * p.n_out;
-      const uint32_t tb = tmem + (static_cast<uint32_t>(lane_base) << 16) + acc * BN_MMA;
       if (EPI == kSiluGated) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -457,9 +616,27 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The gated weights (E x [F gate rows; F up rows] x Kdim) seen as 4-D:
+// (k, row in a 16-row group, gate or up (F rows apart), group).  Only gate
+// groups are addressed, so the last group plus F stays inside the tensor.
+bool make_gate_up_map(CUtensorMap* m, const void* W, int E, int F, int Kdim) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || F % WB_BOX != 0) return false;
+  const uint64_t row = static_cast<uint64_t>(Kdim) * 2;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(Kdim), static_cast<cuuint64_t>(WB_BOX), 2,
+                              static_cast<cuuint64_t>(F) * (2 * E - 1) / WB_BOX};
+  const cuuint64_t strides[3] = {row, row * F, row * WB_BOX};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(WB_BOX), 2u,
+                             static_cast<cuuint32_t>(BMC / (2 * WB_BOX))};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(W), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int EPI, bool GATHER>
-cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params& p, int clusters,
-                       cudaStream_t s) {
+cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& gu,
+                       const TokMaps& tok, const Params& p, int clusters, cudaStream_t s) {
   static std::mutex mu;
   static int resident[64] = {};    // pairs that fit on the device at once (0: not asked yet)
   int dev = 0;
@@ -500,7 +677,7 @@ cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params&
   }
   if (clusters > fit) clusters = fit;
   return launch_k(grouped_gemm_pair_kernel<EPI, GATHER>, dim3(2 * clusters), dim3(THREADS),
-                  kSmemBytes, s, pdl_enabled(), 2, a, b, p);
+                  kSmemBytes, s, pdl_enabled(), 2, a, b, gu, tok, p);
 }
 
 }  // namespace
@@ -508,13 +685,27 @@ cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const Params&
 cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* W,
                                 const int* offsets, int E, int Kdim, int N, int w_rows_per_expert,
                                 const float* bias, void* C, unsigned int* err, cudaStream_t s,
-                                const int* gather_perm, int gather_K, int gather_rows) {
-  CUtensorMap ma, mb;
+                                const int* gather_perm, int gather_K, int gather_rows,
+                                int swap_max) {
+  CUtensorMap ma, mb, mgu;
+  TokMaps tok;
   const bool gather = gather_perm != nullptr;
+  if (swap_max < 0 || swap_max > kSwapMax) return cudaErrorInvalidValue;
   if (!make_map(&ma, A, static_cast<uint64_t>(gather ? gather_rows : a_rows),
                 static_cast<uint64_t>(Kdim), gather ? 1u : 128u) ||
       !make_map(&mb, W, static_cast<uint64_t>(E) * w_rows_per_expert, static_cast<uint64_t>(Kdim)))
     return cudaErrorInvalidValue;
+  // swapped tails: the gated staging needs F % 16 == 0 (whole 16-row groups)
+  if (gather || (act == kSiluGated && N % WB_BOX != 0)) swap_max = 0;
+  mgu = mb;
+  for (int j = 0; j < 4; ++j) tok.m[j] = ma;
+  if (swap_max > 0) {
+    for (int j = 0; j < 4; ++j)
+      if (!make_map(&tok.m[j], A, static_cast<uint64_t>(a_rows), static_cast<uint64_t>(Kdim),
+                    8u << j))
+        return cudaErrorInvalidValue;
+    if (act == kSiluGated && !make_gate_up_map(&mgu, W, E, N, Kdim)) return cudaErrorInvalidValue;
+  }
   Params p;
   p.perm = gather_perm;
   p.K = gather_K;
@@ -527,19 +718,20 @@ cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* 
   p.out = static_cast<__nv_bfloat16*>(C);
   p.bias = bias;
   p.err = err;
+  p.swap_max = swap_max;
   const int bn_out = (act == kSiluGated) ? 128 : 256;
   const long long tiles_bound =
       (static_cast<long long>(a_rows) / BMP + E) * ((N + bn_out - 1) / bn_out);
   const int max_clusters = num_sms() / 2;
   const int clusters = static_cast<int>(tiles_bound < max_clusters ? tiles_bound : max_clusters);
   if (gather) {
-    if (act == kSiluGated) return launch_epi<kSiluGated, true>(ma, mb, p, clusters, s);
-    if (act == kReluBias) return launch_epi<kReluBias, true>(ma, mb, p, clusters, s);
+    if (act == kSiluGated) return launch_epi<kSiluGated, true>(ma, mb, mgu, tok, p, clusters, s);
+    if (act == kReluBias) return launch_epi<kReluBias, true>(ma, mb, mgu, tok, p, clusters, s);
     return cudaErrorInvalidValue;
   }
-  if (act == kSiluGated) return launch_epi<kSiluGated, false>(ma, mb, p, clusters, s);
-  if (act == kReluBias) return launch_epi<kReluBias, false>(ma, mb, p, clusters, s);
-  return launch_epi<kBias, false>(ma, mb, p, clusters, s);
+  if (act == kSiluGated) return launch_epi<kSiluGated, false>(ma, mb, mgu, tok, p, clusters, s);
+  if (act == kReluBias) return launch_epi<kReluBias, false>(ma, mb, mgu, tok, p, clusters, s);
+  return launch_epi<kBias, false>(ma, mb, mgu, tok, p, clusters, s);
 }
 
 }  // namespace moe

@@ -99,12 +99,14 @@ cudaError_t launch_gemm_tc(int act, const void* A, int a_rows, const void* W, co
                            const int* gather_perm = nullptr, int gather_K = 0,
                            int gather_rows = 0);
 
-// Same GEMM on CTA pairs (tcgen05 cta_group::2, 256-row tiles).
+// Same GEMM on CTA pairs (tcgen05 cta_group::2, 256-row tiles).  An expert's
+// last row block of at most swap_max rows (0..255; 0: never) runs as a
+// swapped-operand tile whose N is the block's rows rounded up to 16.
 cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* W,
                                 const int* offsets, int E, int Kdim, int N, int w_rows_per_expert,
                                 const float* bias, void* C, unsigned int* err, cudaStream_t s,
                                 const int* gather_perm = nullptr, int gather_K = 0,
-                                int gather_rows = 0);
+                                int gather_rows = 0, int swap_max = 0);
 
 int num_sms();
 unsigned long long kernel_launches();   // accepted launches so far (note_launch)

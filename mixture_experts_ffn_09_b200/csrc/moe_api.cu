@@ -27,6 +27,7 @@ namespace {
 thread_local std::string g_last_error;
 
 std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
+std::atomic<int> g_tail_swap{MOE_TAIL_SWAP_DEFAULT};
 std::atomic<int> g_fused_gather{0};
 std::atomic<int> g_pdl{0};   // programmatic dependent launch: opt-in
 std::atomic<int> g_debug_sync_ms{0};   // > 0: bounded wait after every kernel of a forward
@@ -46,7 +47,7 @@ cudaError_t launch_gemm_bf16(int act, const void* A, int a_rows, const void* W,
                     (mode == MOE_GEMM_AUTO && static_cast<long long>(T) * K >= 512LL * E);
   if (pair)
     return moe::launch_gemm_tc_pair(act, A, a_rows, W, offsets, E, Kdim, N, w_rows, bias, C, err, s,
-                                    gather_perm, K, T);
+                                    gather_perm, K, T, g_tail_swap.load());
   return moe::launch_gemm_tc(act, A, a_rows, W, offsets, E, static_cast<long long>(T) * K, Kdim, N,
                              w_rows, bias, C, err, s, gather_perm, K, T);
 }
@@ -305,6 +306,11 @@ int moe_set_pdl(int on) { return g_pdl.exchange(on ? 1 : 0); }
 int moe_set_gemm_mode(int mode) {
   if (mode != MOE_GEMM_AUTO && mode != MOE_GEMM_1SM && mode != MOE_GEMM_2SM) return -1;
   return g_gemm_mode.exchange(mode);
+}
+
+int moe_set_tail_swap(int max_rows) {
+  if (max_rows < 0 || max_rows > MOE_TAIL_SWAP_MAX) return -1;
+  return g_tail_swap.exchange(max_rows);
 }
 
 const char* moe_last_error(void) { return g_last_error.c_str(); }

@@ -381,6 +381,15 @@ def set_gemm_mode(mode: int) -> int:
     return prev
 
 
+def set_tail_swap(max_rows: int) -> int:
+    """An expert's last CTA-pair tile of at most max_rows rows (0..128)
+    runs with swapped operands; 0 turns it off.  Returns the previous value."""
+    prev = int(lib().moe_set_tail_swap(int(max_rows)))
+    if prev < 0:
+        raise ValueError(f"tail swap rows out of range: {max_rows}")
+    return prev
+
+
 def set_pdl(on: bool) -> bool:
     """Programmatic dependent launch between a forward's kernels (default
     off; see moe_set_pdl in include/moe.h); returns the previous setting."""

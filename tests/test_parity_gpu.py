@@ -150,6 +150,17 @@ def gemm_mode(request):
 MODES = [1, 2]   # one CTA per tile / CTA pairs (the automatic choice is covered by the workloads)
 
 
+@pytest.fixture
+def tail_swap(request):
+    from mixture_experts_ffn_09_b200 import moe
+    prev = moe.set_tail_swap(request.param)
+    yield request.param
+    moe.set_tail_swap(prev)
+
+
+TAIL_SWAPS = [0, 32, 128]   # off / tails of at most 32 rows / the default (and the maximum)
+
+
 @pytest.mark.parametrize("gemm_mode", MODES, indirect=True)
 @pytest.mark.parametrize("T,D,F,E,K,act,dtype", CASES)
 def test_shapes_and_edges(T, D, F, E, K, act, dtype, gemm_mode):
@@ -165,12 +176,17 @@ def test_shapes_and_edges(T, D, F, E, K, act, dtype, gemm_mode):
 TAIL_COUNTS = [1, 64, 65, 127, 128, 129, 255, 256, 257, 383, 384, 385]
 
 
+@pytest.mark.parametrize("tail_swap", TAIL_SWAPS, indirect=True)
 @pytest.mark.parametrize("gemm_mode", MODES, indirect=True)
 @pytest.mark.parametrize("act", ["silu_gated", "relu"])
-def test_tile_tails_every_boundary(act, gemm_mode):
+def test_tile_tails_every_boundary(act, gemm_mode, tail_swap):
     """Token t is steered to a chosen expert (a dominant router column), so
     every expert gets one of TAIL_COUNTS rows; each tile shape and tail is
-    then compared with the oracle on every token."""
+    then compared with the oracle on every token.  On the pair GEMM the
+    counts put tails on both sides of every swap threshold tested and of
+    every swapped N (tails of 1, 64, 65, 127, 128, 129 and 255 rows)."""
+    if gemm_mode == 1 and tail_swap != 128:
+        pytest.skip("the tail swap applies to the pair GEMM only")
     E, D, F = len(TAIL_COUNTS), 128, 192
     T = sum(TAIL_COUNTS)
     d = dict(synth.random_case(77, T, D, F, E, act=act, dtype="bf16", weight_std=0.05))
@@ -474,11 +490,15 @@ def _random_shapes(n, seed):
     return out
 
 
+@pytest.mark.parametrize("tail_swap", [32, 128], indirect=True)
 @pytest.mark.parametrize("T,D,F,E,K,act,dtype,mode", _random_shapes(12, 2026))
-def test_random_shapes_sweep(T, D, F, E, K, act, dtype, mode):
+def test_random_shapes_sweep(T, D, F, E, K, act, dtype, mode, tail_swap):
     """Seeded random layers (token count, widths, expert count, top-k,
-    activation, dtype, GEMM variant): every token against the oracle."""
+    activation, dtype, GEMM variant, tail swap): every token against the
+    oracle."""
     from mixture_experts_ffn_09_b200 import moe
+    if (mode == 1 or dtype == "f32") and tail_swap != 128:
+        pytest.skip("the tail swap applies to the bf16 pair GEMM only")
     prev = moe.set_gemm_mode(mode)
     try:
         d = synth.random_case(3000 + T + E, T, D, F, E, act=act, dtype=dtype,
