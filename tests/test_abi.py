@@ -52,6 +52,29 @@ def test_abi_version_and_strings(L):
     assert moe.status_string(123) == "unknown status"
 
 
+def test_process_wide_settings_validate_on_host(L):
+    """The GEMM settings are host state: each setter returns the previous
+    value, and refuses an out-of-range one without changing anything."""
+    prev = L.moe_set_tail_swap(64)
+    try:
+        assert prev == 128                       # MOE_TAIL_SWAP_DEFAULT
+        assert L.moe_set_tail_swap(129) == -1    # above MOE_TAIL_SWAP_MAX
+        assert L.moe_set_tail_swap(-1) == -1
+        assert L.moe_set_tail_swap(0) == 64
+        assert L.moe_set_tail_swap(128) == 0
+        with pytest.raises(ValueError):
+            moe.set_tail_swap(200)
+        assert moe.set_tail_swap(32) == 128 and moe.set_tail_swap(128) == 32
+    finally:
+        L.moe_set_tail_swap(prev)
+    g = L.moe_set_gemm_mode(2)
+    try:
+        assert L.moe_set_gemm_mode(7) == -1
+        assert L.moe_set_gemm_mode(1) == 2
+    finally:
+        L.moe_set_gemm_mode(g)
+
+
 def _fwd(L, **kw):
     a = dict(x=P, router=P, gu=P, down=P, E=8, K=2, norm=1, act=0, out=P, sel=P, w=P, T=64, D=64,
              F=128, dt=0, rb=None, b1=None, b2=None, logits=None, ws=P, wsb=1 << 40, stream=None)
