@@ -76,3 +76,18 @@ def test_reference_arm_prints_once_under_torchrun():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["unit"] == "tokens/s"
+    one = d["cpu_baseline"]["single_core"]           # a small float32 layer: one core too
+    assert one["cores"] == 1 and one["value"] > 0
+
+
+def test_oracle_rate_repeats_a_quick_batch():
+    """On a batch far quicker than the budget, the sample is the batch
+    repeated, and the rate is tokens over the summed time."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from mixture_experts_ffn_09_b200 import synth
+    w = synth.SILU_SMALL
+    d = synth.make_inputs(w)
+    rate, n, secs = bench.oracle_rate(w, d, 0.4)
+    assert n > w.T and n % w.T == 0 and secs >= 0.1
+    assert rate == pytest.approx(n / secs)
