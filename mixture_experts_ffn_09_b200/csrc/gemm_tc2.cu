@@ -32,7 +32,7 @@
 // computed and not stored.  The exception is an expert's last row block when
 // it holds at most `swap_max` rows (a short tail): that tile runs with the
 // operands swapped.  The weight rows become the MMA's M = 256 and the tail's
-// token rows its N (rounded up to 16, half from each CTA), so the tensor
+// token rows its N (16, 32, 64 or 128; half from each CTA), so the tensor
 // cores do not spend a full 256-row tile on a few rows.  For the gated
 // expert each CTA stages its 64 gate rows and the matching 64 up rows
 // interleaved in groups of 16, so the gate and up values of one feature land
