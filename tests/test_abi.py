@@ -75,6 +75,44 @@ def test_process_wide_settings_validate_on_host(L):
         L.moe_set_gemm_mode(g)
 
 
+C_CALLER = r'''
+#include <stdio.h>
+#include "moe.h"
+int main(void) {
+  size_t ws = moe_ffn_workspace_size(4096, 4096, 14336, 8, 2, MOE_BF16, MOE_ACT_SILU_GATED);
+  int prev = moe_set_tail_swap(64);
+  int back = moe_set_tail_swap(prev);
+  printf("%d %s %zu %d %d\n", moe_abi_version(), moe_status_string(MOE_ERR_SHAPE), ws, prev, back);
+  return 0;
+}
+'''
+
+
+def test_header_serves_a_plain_c_caller(tmp_path):
+    """The boundary is a C ABI: the header compiles as strict C99 without
+    warnings, and a C program links against the library and calls its
+    host-side entry points."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src, exe = tmp_path / "caller.c", tmp_path / "caller"
+    src.write_text(C_CALLER)
+    libdir = os.path.dirname(moe.LIB_PATH)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                        os.path.join(os.path.dirname(libdir), "include"), str(src), "-o", str(exe),
+                        "-L", libdir, "-lmoe", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    abi, *words = out.stdout.split()
+    assert abi == "1" and " ".join(words[:2]) == "unsupported shape"
+    ws, prev, back = (int(v) for v in words[2:])
+    assert ws == moe.workspace_size(4096, 4096, 14336, 8, 2, moe.BF16, "silu_gated")
+    assert prev == 128 and back == 64
+
+
 def _fwd(L, **kw):
     a = dict(x=P, router=P, gu=P, down=P, E=8, K=2, norm=1, act=0, out=P, sel=P, w=P, T=64, D=64,
              F=128, dt=0, rb=None, b1=None, b2=None, logits=None, ws=P, wsb=1 << 40, stream=None)
