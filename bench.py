@@ -89,10 +89,11 @@ class ClockSampler:
              "nvmlClocksEventReasonHwPowerBrakeSlowdown": "hw_power_brake_slowdown",
              "nvmlClocksEventReasonDisplayClockSetting": "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.01, pci_bus_id: str = None):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period_s
         self.device_index = device_index
+        self.pci_bus_id = pci_bus_id      # NVML numbers GPUs without CUDA_VISIBLE_DEVICES
         self._stop = threading.Event()
         self._ready = threading.Event()
         self.ok = False
@@ -104,7 +105,14 @@ class ClockSampler:
         try:
             import pynvml as N
             N.nvmlInit()
-            h = N.nvmlDeviceGetHandleByIndex(self.device_index)
+            h = None
+            if self.pci_bus_id:
+                try:
+                    h = N.nvmlDeviceGetHandleByPciBusId(self.pci_bus_id)
+                except Exception:
+                    h = None
+            if h is None:
+                h = N.nvmlDeviceGetHandleByIndex(self.device_index)
             self.max_mhz = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
             self.ok = True
         except Exception:
@@ -139,6 +147,16 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
                 "samples": len(self.samples)}
+
+
+def cuda_pci_bus_id(index: int):
+    """'DDDDDDDD:BB:DD.0' of a CUDA device, the form NVML looks GPUs up by."""
+    try:
+        import torch
+        p = torch.cuda.get_device_properties(index)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        return None
 
 
 # ----------------------------------------------------------- accounting
@@ -403,7 +421,7 @@ def run_ours(args, w):
         import torch.distributed as dist
         dist.barrier()
     wd.sync("before the timed region")
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(local, pci_bus_id=cuda_pci_bus_id(local))
     clocks.start()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
