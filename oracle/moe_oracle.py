@@ -46,11 +46,14 @@ Routing extensions ("Mixture of experts", dewml.dev, "Router behavior" and
 * capacity_factor: each sequence of L tokens keeps
   floor(max(ceil(L*K/E)*cf, cf)) slots per expert, the first ones in token
   order; a dropped slot contributes nothing and nothing is renormalised;
-* balancing statistics of a batch from the scores and the dense gate.
+* balancing statistics of a batch from the scores and the gate, the gate
+  being each token's top-k selection renormalised to sum to one.
 
 Parity status: every function here is pinned by the CPU tests in
 ``tests/test_oracle_pins.py`` (worked example, closed forms, invariants,
-brute force, library special cases).  The sources' own seeded outputs (Flax
+brute force, library special cases) and ``tests/test_oracle_ext_pins.py``
+(the routing extensions: hand-worked cases, independent formulations,
+planted mutants).  The sources' own seeded outputs (Flax
 PRNG, mojolearn's generator) cannot be reproduced and are not claimed.
 """
 from __future__ import annotations
@@ -305,16 +308,23 @@ def capacity_keep(idx, E: int, capacity_factor: float, seq_len: int = 0, active=
 
 def balance_stats(scores, idx, weights):
     """The four balancing objectives of ES-MoE's API page ("Balancing
-    objectives") on one batch: probs = the router's scores (T, E), gate =
-    the routing weights scattered to (T, E).
+    objectives") on one batch.  probs = the router's scores (T, E); gate =
+    the top-k selection renormalised (the page's definition), i.e. each
+    token's kept routing weights divided by their sum and scattered to
+    (T, E).  The gate is renormalised whether or not norm_topk_prob was set
+    for the output weights; slots with weight 0 (dropped by the threshold)
+    stay 0.
       switch       = E * sum_i mean(probs)_i * mean(gate > 0)_i
       gshard       = E * sum_i u_i^2, u = mean(gate) normalised to sum to one
       master       = (1/E) * sum_i (u_i - 1/E)^2
       gshard_probs = E * sum_i v_i^2, v = mean(probs) normalised"""
     p = _f64(scores)
     T, E = p.shape
+    w = _f64(weights)
+    tot = w.sum(axis=-1, keepdims=True)
+    w_renorm = np.divide(w, tot, out=np.zeros_like(w), where=tot > 0)
     gate = np.zeros((T, E))
-    np.put_along_axis(gate, np.asarray(idx, dtype=np.int64), _f64(weights), axis=1)
+    np.put_along_axis(gate, np.asarray(idx, dtype=np.int64), w_renorm, axis=1)
     mp = p.mean(axis=0)
     mg = gate.mean(axis=0)
     frac = (gate > 0).mean(axis=0)

@@ -181,16 +181,61 @@ def test_capacity_dropped_slots_add_nothing():
 
 
 # ------------------------------------------------------------- balance
-def test_balance_closed_forms():
+# ES-MoE API page, "Balancing objectives": probs is the router's full score
+# matrix, gate the top-k selection renormalised, both (batch, E); u is a
+# per-expert mean normalised to sum to one.  The hand-worked cases below use
+# fractional gates (so mean(gate > 0) != mean(gate)) and sigmoid scores
+# (whose per-expert means do not sum to one).
+
+# Case A: E=3, two tokens, K=2.  Token 0 scores [0.5, 0.3, 0.2] keeps experts
+# 0, 1 with renormalised gate [5/8, 3/8, 0]; token 1 scores [0.1, 0.3, 0.6]
+# keeps 2, 1 with gate [0, 1/3, 2/3].
+#   mean(probs)    = [0.3, 0.3, 0.4]
+#   mean(gate > 0) = [1/2, 1, 1/2]  -> switch = 3 * (0.15 + 0.3 + 0.2) = 1.95
+#   u = mean(gate) = [5/16, 17/48, 1/3] (sums to one) -> gshard = 3 * 770/2304
+#   master = (gshard - 1) / 9 = 1/3456;  gshard_probs = 3 * 0.34 = 1.02
+CASE_A = dict(probs=[[0.5, 0.3, 0.2], [0.1, 0.3, 0.6]], idx=[[0, 1], [2, 1]],
+              vals=[[0.5, 0.3], [0.6, 0.3]],
+              expect={"switch": 1.95, "gshard": 2310 / 2304, "master": 1 / 3456,
+                      "gshard_probs": 1.02})
+# Case B: sigmoid scores, E=2, K=1.  Scores [0.9, 0.5] and [0.7, 0.1]: both
+# tokens keep expert 0 with gate 1.
+#   mean(probs) = [0.8, 0.3] (sum 1.1) -> v = [8/11, 3/11],
+#   gshard_probs = 2 * 73/121;  switch = 2 * (0.8 * 1 + 0.3 * 0) = 1.6;
+#   u = [1, 0] -> gshard = 2, master = ((1/2)^2 + (1/2)^2) / 2 = 1/4
+CASE_B = dict(probs=[[0.9, 0.5], [0.7, 0.1]], idx=[[0], [0]], vals=[[0.9], [0.7]],
+              expect={"switch": 1.6, "gshard": 2.0, "master": 0.25, "gshard_probs": 146 / 121})
+
+
+def _balance_pins_pass(fn):
+    """The balance pins of this file, run against a (possibly mutated)
+    balance function."""
+    ok = []
+    for case in (CASE_A, CASE_B):
+        p, idx, vals = (np.array(case[k], dtype=np.float64) for k in ("probs", "idx", "vals"))
+        idx = idx.astype(np.int64)
+        # the gate is the renormalised selection: raw kept scores (norm off)
+        # and renormalised weights (norm on) give the same statistics
+        for w in (vals, O.routing_weights(vals, True)):
+            b = fn(p, idx, w)
+            ok.append(all(abs(b[k] - v) <= 1e-9 * max(1.0, abs(v)) for k, v in case["expect"].items()))
+    # the closed forms of a uniform router and of a collapsed one
     E, T = 4, 8
-    p = np.full((T, E), 1.0 / E)
-    idx = (np.arange(T) % E)[:, None]                      # each expert picked by T/E tokens
-    b = O.balance_stats(p, idx, np.ones((T, 1)))
-    assert b == pytest.approx({"switch": 1.0, "gshard": 1.0, "master": 0.0, "gshard_probs": 1.0})
-    idx1 = np.zeros((T, 1), dtype=np.int64)                # everything on expert 0
-    b1 = O.balance_stats(p, idx1, np.ones((T, 1)))
-    assert b1["gshard"] == pytest.approx(E) and b1["master"] == pytest.approx((E - 1) / E ** 2)
-    assert b1["switch"] == pytest.approx(E * (1.0 / E) * 1.0)
+    u = np.full((T, E), 1.0 / E)
+    b = fn(u, (np.arange(T) % E)[:, None], np.ones((T, 1)))
+    ok.append(all(abs(b[k] - v) <= 1e-12 for k, v in
+                  {"switch": 1.0, "gshard": 1.0, "master": 0.0, "gshard_probs": 1.0}.items()))
+    b = fn(u, np.zeros((T, 1), dtype=np.int64), np.ones((T, 1)))
+    ok.append(abs(b["gshard"] - E) <= 1e-12 and abs(b["master"] - (E - 1) / E ** 2) <= 1e-12
+              and abs(b["switch"] - 1.0) <= 1e-12)
+    # a slot with weight 0 (dropped by the threshold) is not a selection
+    b = fn(np.array([[0.6, 0.4]]), np.array([[0, 1]]), np.array([[1.0, 0.0]]))
+    ok.append(abs(b["switch"] - 2 * 0.6) <= 1e-12 and abs(b["gshard"] - 2.0) <= 1e-12)
+    return all(ok)
+
+
+def test_balance_hand_worked_cases():
+    assert _balance_pins_pass(O.balance_stats)
 
 
 def test_balance_master_is_gshard_minus_one_over_e_squared():
@@ -199,6 +244,68 @@ def test_balance_master_is_gshard_minus_one_over_e_squared():
     b = O.balance_stats(r["probs"], r["selected_experts"], r["routing_weights"])
     assert b["master"] == pytest.approx((b["gshard"] - 1) / 8 ** 2, rel=1e-12)
     assert 1.0 <= b["gshard"] <= 8.0 and 1.0 <= b["gshard_probs"] <= 8.0
+
+
+@pytest.mark.parametrize("score", [O.SCORE_SOFTMAX, O.SCORE_SIGMOID])
+def test_balance_does_not_depend_on_norm_topk_prob(score):
+    """The gate is renormalised by definition, so the forward's statistics
+    are the same with and without the output weights' renormalisation."""
+    d = _case(12, 40, 8, 6, 6)
+    kw = dict(score=score)
+    a = O.moe_ffn_forward_ext(d["x"], d["router"], d["gate_up_proj"], d["down_proj"], K=3,
+                              norm_topk_prob=True, **kw)["balance"]
+    b = O.moe_ffn_forward_ext(d["x"], d["router"], d["gate_up_proj"], d["down_proj"], K=3,
+                              norm_topk_prob=False, **kw)["balance"]
+    for k in a:
+        assert a[k] == pytest.approx(b[k], rel=1e-12), k
+
+
+def test_balance_mutants_are_caught():
+    """Plausible misreadings of the objectives, each of which the pins above
+    must reject."""
+    def gate_of(p, idx, w, renorm=True):
+        w = np.asarray(w, dtype=np.float64)
+        if renorm:
+            w = w / w.sum(-1, keepdims=True)
+        g = np.zeros(np.shape(p))
+        np.put_along_axis(g, np.asarray(idx, dtype=np.int64), w, axis=1)
+        return g
+
+    def stats(p, g, switch_frac=None, norm_v=True, master_scale=1.0):
+        p = np.asarray(p, dtype=np.float64)
+        E = p.shape[1]
+        mp, mg = p.mean(0), g.mean(0)
+        frac = (g > 0).mean(0) if switch_frac is None else switch_frac
+        u = mg / mg.sum()
+        v = mp / mp.sum() if norm_v else mp
+        return {"switch": E * float((mp * frac).sum()), "gshard": E * float((u * u).sum()),
+                "master": master_scale * float(((u - 1 / E) ** 2).sum() / E),
+                "gshard_probs": E * float((v * v).sum())}
+
+    def switch_on_mean_gate(p, idx, w):
+        g = gate_of(p, idx, w)
+        return stats(p, g, switch_frac=g.mean(0))
+
+    def gshard_probs_unnormalised(p, idx, w):
+        return stats(p, gate_of(p, idx, w), norm_v=False)
+
+    def gate_not_renormalised(p, idx, w):
+        return stats(p, gate_of(p, idx, w, renorm=False))
+
+    def master_without_one_over_e(p, idx, w):
+        return stats(p, gate_of(p, idx, w), master_scale=np.shape(p)[1])
+
+    def gshard_reads_probs(p, idx, w):
+        r = stats(p, gate_of(p, idx, w))
+        r["gshard"] = r["gshard_probs"]
+        return r
+
+    # the helpers reproduce the oracle when unmutated, so each mutant differs
+    # from it in exactly one place
+    assert _balance_pins_pass(lambda p, idx, w: stats(p, gate_of(p, idx, w)))
+    for fn in (switch_on_mean_gate, gshard_probs_unnormalised, gate_not_renormalised,
+               master_without_one_over_e, gshard_reads_probs):
+        assert not _balance_pins_pass(fn), fn.__name__
 
 
 def test_ext_forward_without_extensions_is_the_plain_forward():
