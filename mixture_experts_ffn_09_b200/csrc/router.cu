@@ -208,16 +208,29 @@ __global__ void __launch_bounds__(kWarps * 32) router_topk_kernel(RouteArgs a) {
         if (k == 0 || sh >= a.dyn_threshold) ksum += sh;
       }
     const float denom = a.norm ? (psum + 1e-9f) : 1.f;
-    for (int k = lane; k < K; k += 32) {
-      const int e = sel[k];
+    auto weight = [&](int k, bool& keep) {
       const float p = selv[k];
       float w = a.norm ? p / denom : p;
-      bool keep = true;
+      keep = true;
       if (a.dyn_threshold > 0.f) {
         const float sh = p / psum;
         keep = k == 0 || sh >= a.dyn_threshold;
         w = keep ? sh / ksum : 0.f;
       }
+      return w;
+    };
+    // the balance statistics read the selection renormalised to sum to one
+    // (whether or not the output weights are): gate = w / sum of the kept w
+    float wsum = 0.f;
+    if (a.bal_partial)
+      for (int k = 0; k < K; ++k) {
+        bool kk;
+        wsum += weight(k, kk);
+      }
+    for (int k = lane; k < K; k += 32) {
+      const int e = sel[k];
+      bool keep;
+      const float w = weight(k, keep);
       const size_t o = static_cast<size_t>(t) * K + k;
       if (a.sel64) a.sel64[o] = e;
       if (a.wout) a.wout[o] = w;
@@ -226,8 +239,9 @@ __global__ void __launch_bounds__(kWarps * 32) router_topk_kernel(RouteArgs a) {
       if (a.slot_kept) a.slot_kept[o] = keep ? 1 : 0;
       if (keep && a.blockcounts) atomicAdd(&hist[e], 1);
       if (a.bal_partial) {
-        bal[E + e] += w;
-        bal[2 * E + e] += w > 0.f ? 1.f : 0.f;
+        const float g = wsum > 0.f ? w / wsum : 0.f;
+        bal[E + e] += g;
+        bal[2 * E + e] += g > 0.f ? 1.f : 0.f;
       }
     }
     __syncwarp();

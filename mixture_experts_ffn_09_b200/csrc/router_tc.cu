@@ -497,19 +497,26 @@ __global__ void __launch_bounds__(THREADS, 1)
         bp[e] = acc;
       }
       asm volatile("bar.sync 2, 128;" ::: "memory");
+      // the row's gate: its kept weights renormalised to sum to one (the
+      // selection renormalised, whether or not the output weights are)
       for (int e = 0; e < E; ++e) lrow[e] = 0.f;
       if (valid) {
         if (p.K <= 8) {
+          float wsum = 0.f;
+          for (int k = 0; k < p.K; ++k)
+            if (!(sel_e[k * BM + row] & kDroppedBit)) wsum += sel_p[k * BM + row];
           for (int k = 0; k < p.K; ++k) {
             const int e = sel_e[k * BM + row];
-            if (!(e & kDroppedBit)) lrow[e] = sel_p[k * BM + row];
+            if (!(e & kDroppedBit)) lrow[e] = wsum > 0.f ? sel_p[k * BM + row] / wsum : 0.f;
           }
         } else {
+          const float* wk = (p.w32 ? p.w32 : p.wout) + static_cast<size_t>(t) * p.K;
+          float wsum = 0.f;
+          for (int k = 0; k < p.K; ++k) wsum += wk[k];   // dropped slots hold 0
           for (int k = 0; k < p.K; ++k) {
             const size_t o = static_cast<size_t>(t) * p.K + k;
             const int e = p.idx32 ? p.idx32[o] : static_cast<int>(p.sel64[o]);
-            const float w = p.w32 ? p.w32[o] : p.wout[o];
-            if (e < E) lrow[e] = w;
+            if (e < E) lrow[e] = wsum > 0.f ? wk[k] / wsum : 0.f;
           }
         }
       }

@@ -111,6 +111,22 @@ def test_scores_and_selection_bias(T, D, F, E, K, dtype, score, biased):
     check_ext(d, E, K, True, "silu_gated", dtype, score=score, sel_bias=bias)
 
 
+@pytest.mark.parametrize("T,D,F,E,K,dtype", CASES + [(256, 64, 64, 16, 10, "bf16"),
+                                                      (256, 64, 64, 16, 10, "f32")])
+@pytest.mark.parametrize("score", ["softmax", "sigmoid"])
+def test_balance_with_norm_topk_prob_off(T, D, F, E, K, dtype, score):
+    """With norm_topk_prob off the output weights are the raw kept scores,
+    but the balance statistics still read the renormalised selection (ES-MoE
+    API page, "Balancing objectives").  K = 10 takes the routers'
+    round-per-choice path."""
+    d = synth.random_case(400 + T + K, T, D, F, E, dtype=dtype,
+                          weight_std=0.3 if dtype == "f32" else 0.05)
+    g = check_ext(d, E, K, False, "silu_gated", dtype, score=score)
+    # the raw kept scores do not sum to one, so a gate that was not
+    # renormalised would give other statistics
+    assert np.abs(g["w"].sum(1) - 1.0).max() > 1e-3
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("th", [0.15, 0.3, 0.9])
 def test_dynamic_threshold(dtype, th):
