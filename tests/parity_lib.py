@@ -48,15 +48,20 @@ def host_views(d: dict) -> dict:
 
 
 def to_device(d: dict, device="cuda"):
+    """Device copies of the generator's (read-only) arrays; the host views
+    are only read, so torch's warning about non-writable arrays is muted."""
+    import warnings
     import torch
     out = {}
-    for k, v in d.items():
-        if v is None:
-            out[k] = None
-        elif v.dtype == np.uint16:
-            out[k] = torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).view(torch.bfloat16).to(device)
-        else:
-            out[k] = torch.from_numpy(np.ascontiguousarray(v)).to(device)
+    with warnings.catch_warnings():
+        warnings.filterwarnings("ignore", message="The given NumPy array is not writable")
+        for k, v in d.items():
+            if v is None:
+                out[k] = None
+            elif v.dtype == np.uint16:
+                out[k] = torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).view(torch.bfloat16).to(device)
+            else:
+                out[k] = torch.from_numpy(np.ascontiguousarray(v)).to(device)
     return out
 
 
@@ -129,9 +134,28 @@ def oracle_out_for(h: dict, tokens, sel, K: int, norm: bool, act: str):
     return O.moe_ffn_given_routing(x, sel, w, h["gate_up_proj"], h["down_proj"], act, h["b1"], h["b2"])
 
 
-def sample_tokens(sel_ref: np.ndarray, E: int, n: int, seed: int = 0) -> np.ndarray:
+def tail_tokens(sel: np.ndarray, E: int) -> dict:
+    """Tokens whose rows sit in each expert's last row blocks.
+
+    The permutation sorts an expert's rows by token index, so the expert's
+    last rows belong to its highest-index tokens.  For every expert this
+    returns the token of its last row, and the first token of its last
+    128-row and last 256-row block (the one-CTA and CTA-pair tiles: a pair
+    GEMM's short last block runs with swapped operands).  Keyed by expert."""
+    out = {}
+    for e in range(E):
+        toks = np.nonzero((sel == e).any(1))[0]
+        n = len(toks)
+        if n:
+            out[e] = sorted({int(toks[-1]), int(toks[(n - 1) // 128 * 128]),
+                             int(toks[(n - 1) // 256 * 256])})
+    return out
+
+
+def sample_tokens(sel_ref: np.ndarray, E: int, n: int, seed: int = 0, tails=None) -> np.ndarray:
     """A seeded token subset that covers every expert selected anywhere,
-    plus the first and last token, topped up at random to n tokens."""
+    plus the first and last token and the given tail tokens (see
+    tail_tokens), topped up at random to n tokens."""
     rng = np.random.default_rng(seed)
     T = sel_ref.shape[0]
     order = rng.permutation(T)
@@ -140,6 +164,8 @@ def sample_tokens(sel_ref: np.ndarray, E: int, n: int, seed: int = 0) -> np.ndar
         hit = order[(sel_ref[order] == e).any(1)]
         if len(hit):
             chosen.add(int(hit[0]))
+    for toks in (tails or {}).values():
+        chosen.update(toks)
     for t in order:
         if len(chosen) >= n:
             break

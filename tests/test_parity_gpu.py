@@ -84,9 +84,19 @@ def _sampled_full_size(w, n_sample):
     r = PL.oracle_route(h, w.K, w.norm_topk_prob)
     clear = PL.check_routing(g, r, w.K, w.norm_topk_prob)
     assert clear.mean() > 0.99
-    tok = PL.sample_tokens(r["selected_experts"], w.E, n_sample)
+    # the sample reaches every expert's last row blocks (on the GPU's own
+    # selection, which decides the sorted rows), so the tail tiles - swapped
+    # on the CTA-pair GEMM - are checked at full K depth
+    tails = PL.tail_tokens(g["sel"], w.E)
+    tok = PL.sample_tokens(r["selected_experts"], w.E, n_sample, tails=tails)
     ref = PL.oracle_out_for(h, tok, g["sel"][tok], w.K, w.norm_topk_prob, w.act)
     PL.check_out(g["out"][tok], ref, w.dtype)
+    tail_set = sorted({t for v in tails.values() for t in v})
+    assert set(tail_set) <= set(tok.tolist())
+    pos = {int(t): i for i, t in enumerate(tok)}
+    ti = [pos[t] for t in tail_set]
+    PL.check_out(g["out"][tok][ti], ref[ti], w.dtype,
+                 f"tail-block tokens of every expert ({len(tail_set)} tokens)")
     # every token's output is finite and no row was left unwritten
     assert np.isfinite(g["out"]).all()
     return g, r
