@@ -229,10 +229,22 @@ MOE_API moe_status_t moe_route_ex(const void* x, const void* router, const float
  * before anything is launched (for bf16 that covers e.g. T=32 tokens with
  * D=4096, F=14336, E=8, K=8).  No cudaMalloc / cudaFree is called.
  *
- * The first call on a device looks up the array's device address (with that
- * device current); make that first call before any stream capture.  All
- * calls share the one array and it keeps the previous call's contents; no
- * part of it has to start at zero, since each call writes every scratch
+ * The first call on a device does a one-time host-side set-up with that
+ * device current: it reads the device's attributes and looks up the device
+ * addresses of the array and of the library's error word
+ * (cudaGetSymbolAddress).  If the CUDA runtime loads modules lazily, that
+ * lookup is what loads the library's device code, and with it the driver
+ * places the 32 MiB array in device memory.  Later calls reuse what the first
+ * one found.  So make the first call on each device part of the caller's
+ * initialisation, before any stream capture.  This entry point creates no
+ * stream, event or pinned host memory (the other entry points create one
+ * each per device on their first call, for reading the error word during a
+ * stall); the first moe_set_debug_sync wait or moe_device_error_peek on a
+ * device creates them.  A cudaDeviceReset discards what the set-up found:
+ * calls after one, in the same process, are not supported.
+ *
+ * All calls share the one array and it keeps the previous call's contents;
+ * no part of it has to start at zero, since each call writes every scratch
  * element it later reads (pad rows only feed rows that are never stored).
  * Calls whose work overlaps on the GPU (e.g. on two streams at once) race
  * on the array: order them on one stream or with events.

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/moe.h"
+
 namespace moe {
 
 constexpr int kMaxExperts = 256;
@@ -117,5 +119,18 @@ cudaError_t launch_bounded_wait_probe(unsigned long long timeout_ns, unsigned in
 
 // Sets the message moe_last_error() returns on this host thread.
 void set_last_error(const char* msg);
+
+// The whole forward behind moe_ffn_forward_ex.  with_aux = false skips the
+// per-device host bookkeeping (a stream, an event and a pinned host word
+// for reading the error word during a stall), so the call allocates
+// nothing; the no-allocation entry point uses that.
+moe_status_t ffn_forward_impl(const void* x, const void* router, const void* gate_up_proj,
+                              const void* down_proj, int E, int K, int norm_topk_prob,
+                              moe_act_t act, void* out, int64_t* selected_experts,
+                              float* routing_weights, int64_t T, int64_t D, int64_t F,
+                              moe_dtype_t dt, const float* router_bias, const float* b1,
+                              const float* b2, float* router_logits, void* workspace,
+                              size_t workspace_bytes, const moe_route_opts_t* opts, void* stream,
+                              bool with_aux);
 
 }  // namespace moe

@@ -79,8 +79,12 @@ struct DevInfo {
   int sms = 0;
   int major = 0, minor = 0;
   unsigned int* err = nullptr;
-  // created once, so that reading the error word during a stall needs no
-  // call that could wait for the device
+  // Host-side bookkeeping for reading the error word while kernels may be
+  // stalled, made once per device so that such a read needs no call that
+  // could wait for the device.  The ordinary entry points create it on
+  // their first call; the no-allocation entry point never does (it holds a
+  // pinned host word), and the readers create it on first use.
+  bool aux = false;
   cudaStream_t peek_stream = nullptr;
   unsigned int* peek_host = nullptr;
   cudaEvent_t dbg_event = nullptr;
@@ -88,7 +92,21 @@ struct DevInfo {
 std::mutex g_dev_mu;
 DevInfo g_dev[64];
 
-moe_status_t device_info(DevInfo** out) {
+// Creates the device's stream, event and pinned word (g_dev_mu held).
+moe_status_t make_aux(DevInfo& d) {
+  if (d.aux) return MOE_OK;
+  cudaError_t e;
+  if ((e = cudaStreamCreateWithFlags(&d.peek_stream, cudaStreamNonBlocking)) != cudaSuccess ||
+      (e = cudaMallocHost(&d.peek_host, sizeof(unsigned int))) != cudaSuccess ||
+      (e = cudaEventCreateWithFlags(&d.dbg_event, cudaEventDisableTiming)) != cudaSuccess)
+    return cuda_fail(e, "device bookkeeping");
+  d.aux = true;
+  return MOE_OK;
+}
+
+// The current device's attributes and error-word address, checked to be an
+// sm_100 part; with_aux also sets up the bookkeeping above.
+moe_status_t device_info(DevInfo** out, bool with_aux = true) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -106,17 +124,23 @@ moe_status_t device_info(DevInfo** out) {
     if ((e = cudaGetSymbolAddress(&p, g_device_error)) != cudaSuccess)
       return cuda_fail(e, "cudaGetSymbolAddress(error word)");
     d.err = static_cast<unsigned int*>(p);
-    if ((e = cudaStreamCreateWithFlags(&d.peek_stream, cudaStreamNonBlocking)) != cudaSuccess ||
-        (e = cudaMallocHost(&d.peek_host, sizeof(unsigned int))) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&d.dbg_event, cudaEventDisableTiming)) != cudaSuccess)
-      return cuda_fail(e, "device bookkeeping");
     d.init = true;
   }
   if (d.major != 10 || d.minor != 0)
     return fail(MOE_ERR_DEVICE, "device %d is sm_%d%d; libmoe is built for sm_100a", dev, d.major,
                 d.minor);
+  if (with_aux) {
+    const moe_status_t st = make_aux(d);
+    if (st != MOE_OK) return st;
+  }
   *out = &d;
   return MOE_OK;
+}
+
+// The bookkeeping of a device whose DevInfo exists already (made on first use).
+bool ensure_aux(DevInfo* d) {
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  return make_aux(*d) == MOE_OK;
 }
 
 // Polls until `done()` or `ms` milliseconds have passed.
@@ -135,6 +159,7 @@ bool poll_ms(int ms, Done done) {
 bool peek_word(DevInfo* dev, unsigned int* word, int ms) {
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
+  if (!ensure_aux(dev)) return false;
   if (cudaMemcpyAsync(dev->peek_host, dev->err, sizeof(unsigned int), cudaMemcpyDeviceToHost,
                       dev->peek_stream) != cudaSuccess)
     return false;
@@ -149,6 +174,10 @@ bool peek_word(DevInfo* dev, unsigned int* word, int ms) {
 bool debug_wait(DevInfo* dev, cudaStream_t s, const char* stage) {
   const int ms = g_debug_sync_ms.load();
   if (ms <= 0) return true;
+  if (!ensure_aux(dev)) {
+    fail(MOE_ERR_CUDA, "debug sync after %s: could not create its event", stage);
+    return false;
+  }
   if (cudaEventRecord(dev->dbg_event, s) == cudaSuccess &&
       poll_ms(ms, [&] { return cudaEventQuery(dev->dbg_event) != cudaErrorNotReady; }))
     return true;
@@ -408,6 +437,22 @@ moe_status_t moe_ffn_forward_ex(const void* x, const void* router, const void* g
                                 const float* b2, float* router_logits, void* workspace,
                                 size_t workspace_bytes, const moe_route_opts_t* opts,
                                 void* stream) {
+  return moe::ffn_forward_impl(x, router, gate_up_proj, down_proj, E, K, norm_topk_prob, act, out,
+                               selected_experts, routing_weights, T, D, F, dt, router_bias, b1, b2,
+                               router_logits, workspace, workspace_bytes, opts, stream, true);
+}
+
+}  // extern "C"
+
+namespace moe {
+moe_status_t ffn_forward_impl(const void* x, const void* router, const void* gate_up_proj,
+                              const void* down_proj, int E, int K, int norm_topk_prob,
+                              moe_act_t act, void* out, int64_t* selected_experts,
+                              float* routing_weights, int64_t T, int64_t D, int64_t F,
+                              moe_dtype_t dt, const float* router_bias, const float* b1,
+                              const float* b2, float* router_logits, void* workspace,
+                              size_t workspace_bytes, const moe_route_opts_t* opts, void* stream,
+                              bool with_aux) {
   g_last_error.clear();
   moe_status_t st = check_common(T, D, E, K, dt);
   if (st != MOE_OK) return st;
@@ -436,7 +481,7 @@ moe_status_t moe_ffn_forward_ex(const void* x, const void* router, const void* g
     return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", L.total,
                 workspace ? workspace_bytes : static_cast<size_t>(0));
   DevInfo* dev = nullptr;
-  if ((st = device_info(&dev)) != MOE_OK) return st;
+  if ((st = device_info(&dev, with_aux)) != MOE_OK) return st;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -552,6 +597,9 @@ moe_status_t moe_ffn_forward_ex(const void* x, const void* router, const void* g
   if (!debug_wait(dev, s, "combine")) return MOE_ERR_TIMEOUT;
   return MOE_OK;
 }
+}  // namespace moe
+
+extern "C" {
 
 moe_status_t moe_debug_bounded_wait(int timeout_ms, void* stream) {
   g_last_error.clear();

@@ -7,7 +7,10 @@
 //
 // No call here allocates: the array is static, its device address is looked
 // up once per device with cudaGetSymbolAddress, and the work itself is the
-// ordinary moe_ffn_forward with that address as its workspace.
+// ordinary forward with that address as its workspace, run without the host
+// bookkeeping (stream, event, pinned word) the other entry points set up.
+// The addresses cached per device belong to the process's CUDA context: a
+// cudaDeviceReset invalidates them, and calls after one are not supported.
 #include <stdio.h>
 
 #include <mutex>
@@ -70,9 +73,9 @@ extern "C" moe_status_t moe_ffn_forward_noalloc(const void* x, const void* route
   if (need == 0) {
     // invalid sizes: let the ordinary entry point report exactly which
     // argument is wrong (it validates before touching the workspace)
-    return moe_ffn_forward(x, router, gate_up_proj, down_proj, E, K, norm_topk_prob, act, out,
-                           selected_experts, routing_weights, T, D, F, dt, router_bias, b1, b2,
-                           router_logits, nullptr, 0, stream);
+    return moe::ffn_forward_impl(x, router, gate_up_proj, down_proj, E, K, norm_topk_prob, act,
+                                 out, selected_experts, routing_weights, T, D, F, dt, router_bias,
+                                 b1, b2, router_logits, nullptr, 0, nullptr, stream, false);
   }
   if (need > MOE_NOALLOC_SCRATCH_BYTES) {
     char buf[256];
@@ -86,7 +89,8 @@ extern "C" moe_status_t moe_ffn_forward_noalloc(const void* x, const void* route
   void* scratch = nullptr;
   const moe_status_t st = scratch_address(&scratch);
   if (st != MOE_OK) return st;
-  return moe_ffn_forward(x, router, gate_up_proj, down_proj, E, K, norm_topk_prob, act, out,
-                         selected_experts, routing_weights, T, D, F, dt, router_bias, b1, b2,
-                         router_logits, scratch, MOE_NOALLOC_SCRATCH_BYTES, stream);
+  return moe::ffn_forward_impl(x, router, gate_up_proj, down_proj, E, K, norm_topk_prob, act, out,
+                               selected_experts, routing_weights, T, D, F, dt, router_bias, b1, b2,
+                               router_logits, scratch, MOE_NOALLOC_SCRATCH_BYTES, nullptr, stream,
+                               false);
 }

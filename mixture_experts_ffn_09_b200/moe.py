@@ -198,10 +198,10 @@ def _expect(t, shape, name, dtype=None, required=True):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
 
 
 def ffn_forward(x, router, gate_up_proj, down_proj, E: int, K: int, norm_topk_prob: bool, act,
@@ -217,11 +217,11 @@ def ffn_forward(x, router, gate_up_proj, down_proj, E: int, K: int, norm_topk_pr
     if dt in (F32, BF16) and a in (ACT_SILU_GATED, ACT_RELU) and 1 <= K <= E and T > 0:
         wdt = x.dtype
         gu_rows = 2 * F if a == ACT_SILU_GATED else F
+        _expect(x, tuple(x.shape), "x", wdt)
         _expect(router, (E, D), "router", wdt)
         _expect(gate_up_proj, (E, gu_rows, D), "gate_up_proj", wdt)
         _expect(down_proj, (E, D, F), "down_proj", wdt)
         _expect(out, tuple(x.shape), "out", wdt)
-        _expect(x, tuple(x.shape), "x", wdt)
         _expect(selected_experts, (T, K), "selected_experts", torch.int64, False)
         _expect(routing_weights, (T, K), "routing_weights", torch.float32, False)
         _expect(router_bias, (E,), "router_bias", torch.float32, False)
@@ -256,6 +256,7 @@ def ffn_forward_noalloc(x, router, gate_up_proj, down_proj, E: int, K: int, norm
     if dt in (F32, BF16) and a in (ACT_SILU_GATED, ACT_RELU) and 1 <= K <= E and T > 0:
         wdt = x.dtype
         gu_rows = 2 * F if a == ACT_SILU_GATED else F
+        _expect(x, tuple(x.shape), "x", wdt)
         _expect(router, (E, D), "router", wdt)
         _expect(gate_up_proj, (E, gu_rows, D), "gate_up_proj", wdt)
         _expect(down_proj, (E, D, F), "down_proj", wdt)
@@ -274,7 +275,10 @@ def ffn_forward_noalloc(x, router, gate_up_proj, down_proj, E: int, K: int, norm
 
 
 def noalloc_scratch_bytes() -> int:
-    """Size of the static scratch behind ffn_forward_noalloc (32 MiB)."""
+    """Size of the static scratch behind ffn_forward_noalloc: the value of
+    MOE_NOALLOC_SCRATCH_BYTES in include/moe.h (32 MiB).  A CPU test pins it
+    against the library: sizes up to it pass the size check, one byte more
+    of workspace is refused."""
     return 32 << 20
 
 
@@ -302,6 +306,7 @@ def ffn_forward_ex(x, router, gate_up_proj, down_proj, E: int, K: int, norm_topk
     if dt in (F32, BF16) and a in (ACT_SILU_GATED, ACT_RELU) and 1 <= K <= E and T > 0:
         wdt = x.dtype
         gu_rows = 2 * F if a == ACT_SILU_GATED else F
+        _expect(x, tuple(x.shape), "x", wdt)
         _expect(router, (E, D), "router", wdt)
         _expect(gate_up_proj, (E, gu_rows, D), "gate_up_proj", wdt)
         _expect(down_proj, (E, D, F), "down_proj", wdt)
@@ -334,6 +339,7 @@ def route_ex(x, router, K: int, norm_topk_prob: bool, selected_experts, routing_
     E = int(router.shape[0])
     dt = _dtype_code(x)
     if dt in (F32, BF16) and 1 <= K <= E and T > 0:
+        _expect(x, tuple(x.shape), "x", x.dtype)
         _expect(router, (E, D), "router", x.dtype)
         _expect(selected_experts, (T, K), "selected_experts", torch.int64)
         _expect(routing_weights, (T, K), "routing_weights", torch.float32)
@@ -358,6 +364,7 @@ def route(x, router, K: int, norm_topk_prob: bool, selected_experts, routing_wei
     E = int(router.shape[0])
     dt = _dtype_code(x)
     if dt in (F32, BF16) and 1 <= K <= E and T > 0:
+        _expect(x, tuple(x.shape), "x", x.dtype)
         _expect(router, (E, D), "router", x.dtype)
         _expect(selected_experts, (T, K), "selected_experts", torch.int64)
         _expect(routing_weights, (T, K), "routing_weights", torch.float32)

@@ -55,6 +55,7 @@ def _both(d, E, K, act, dtype):
     np.testing.assert_array_equal(s, s_ref)
     np.testing.assert_allclose(w, w_ref, atol=1e-6, rtol=0)
     PL.check_out(o, o_ref, dtype, "no-allocation forward vs workspace forward")
+    return s
 
 
 @pytest.mark.gpu
@@ -79,3 +80,68 @@ def test_noalloc_refuses_sizes_beyond_its_scratch():
     st = L.moe_ffn_forward_noalloc(P, P, P, P, 8, 9, 1, 0, P, None, None, 32, 64, 64, moe.BF16,
                                    None, None, None, None, None)
     assert st == moe.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.gpu
+def test_noalloc_on_the_cta_pair_gemm():
+    """The CTA-pair GEMM over the shared scratch: its short expert tails run
+    with swapped operands (extra token views over the expert-sorted rows),
+    longer tails as padded 256-row tiles whose pad rows hold whatever the
+    previous call left there.  Both kinds, after calls with other shapes."""
+    prev = moe.set_gemm_mode(moe.GEMM_2SM)
+    try:
+        long_tails = synth.random_case(44, 900, 512, 1024, 2, dtype="bf16", weight_std=0.05)
+        short_tails = synth.random_case(45, 600, 256, 384, 6, dtype="bf16", weight_std=0.05)
+        tails = []
+        for d, E in ((long_tails, 2), (short_tails, 6), (long_tails, 2)):
+            sel = _both(d, E, 1, "silu_gated", "bf16")
+            rows = np.bincount(sel.ravel(), minlength=E)
+            tails += [int(r) % 256 for r in rows if r % 256]
+        assert any(1 <= t <= 128 for t in tails), tails      # swapped
+        assert any(129 <= t <= 255 for t in tails), tails    # padded full tile
+    finally:
+        moe.set_gemm_mode(prev)
+
+
+def test_noalloc_scratch_size_edge():
+    """The scratch size the binding reports is the one the library enforces:
+    the largest layer of this shape whose workspace fits gets past the size
+    check, one token more is refused.  The pointers are misaligned on purpose,
+    so a call that passes the size check is rejected on the host before any
+    launch (MOE_ERR_ALIGNMENT; MOE_ERR_CUDA where no GPU is present)."""
+    L = moe.lib()
+    lim = moe.noalloc_scratch_bytes()
+    D, F, E, K = 32, 32, 4, 1
+    lo, hi = 1, 1 << 20                       # workspace(lo) <= lim < workspace(hi)
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        if moe.workspace_size(mid, D, F, E, K, moe.BF16) <= lim:
+            lo = mid
+        else:
+            hi = mid
+    assert lim - moe.workspace_size(lo, D, F, E, K, moe.BF16) <= 8192
+    P = 0x10001
+    for T, refused in ((lo, False), (hi, True)):
+        st = L.moe_ffn_forward_noalloc(P, P, P, P, E, K, 1, 0, P, None, None, T, D, F, moe.BF16,
+                                       None, None, None, None, None)
+        if refused:
+            assert st == moe.MOE_ERR_WORKSPACE and "static scratch" in moe.last_error()
+        else:
+            assert st in (moe.MOE_ERR_ALIGNMENT, moe.MOE_ERR_CUDA, moe.MOE_ERR_DEVICE), st
+
+
+def test_noalloc_rejects_a_non_contiguous_x():
+    """A strided view of x would reach the C ABI as if it were a dense
+    (T, D) matrix; the binding refuses it, as it does for the ordinary
+    entry point."""
+    import torch
+    T, D, F, E, K = 8, 64, 32, 4, 2
+    x = torch.zeros(T, 2 * D, dtype=torch.float32)[:, ::2]
+    assert x.shape == (T, D) and not x.is_contiguous()
+    router = torch.zeros(E, D)
+    gu = torch.zeros(E, 2 * F, D)
+    dn = torch.zeros(E, D, F)
+    out = torch.zeros(T, D)
+    for fn in (moe.ffn_forward_noalloc, moe.ffn_forward):
+        with pytest.raises(ValueError, match="^x must be contiguous"):
+            fn(x, router, gu, dn, E, K, True, "silu_gated", out)
