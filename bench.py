@@ -41,6 +41,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "source": "fallback"}
 NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 L2_BYTES = 126 * 1024 * 1024
+# The configs timed after the headline one in the same run (each with its own
+# inputs, warm-up, timed forwards and per-stage pass).
+EXTRA_WORKLOADS = ("decode_t32_d4096_f14336_e8_k1_bf16", "decode_t32_d4096_f14336_e8_k2_bf16",
+                   "decode_t32_d4096_f14336_e8_k8_bf16",
+                   "fine_grained_t16384_d2048_f1408_e64_k6_zipf_bf16",
+                   "dense_relu_t64_d32_f64_e4_k2_f32", "silu_gated_t64_d64_f128_e8_k2_f32")
 
 
 def load_peaks() -> dict:
@@ -338,6 +344,205 @@ def workload_config(w, world: int) -> dict:
 
 
 # ---------------------------------------------------------------- our arm
+PEAK_FLOP_PER_CLK_PER_SM = 8192     # dense bf16 tcgen05 MMA: 8192 FLOP per SM per clock
+SMS = 148
+SUSTAINED_AFTER_S = 2.0             # a kernel timed inside a loop this long runs power-capped
+
+
+def _readonly_view(a):
+    """torch view of a read-only numpy array that is only ever read (copied
+    to the device or to pinned memory), without torch's writability warning."""
+    import warnings
+    import numpy as np
+    import torch
+    with warnings.catch_warnings():
+        warnings.filterwarnings("ignore", message="The given NumPy array is not writable")
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a))
+
+
+class Layer:
+    """Device buffers of one workload and the forward through the C ABI."""
+
+    def __init__(self, w, d, dev, args, ext_opts=None):
+        import torch
+        from mixture_experts_ffn_09_b200 import moe
+        self.w, self.dev = w, dev
+        up = (lambda a: None if a is None else _readonly_view(a).to(dev))
+        self.x = up(d["x"]).reshape(w.T, w.D)
+        self.router, self.gu, self.dn = up(d["router"]), up(d["gate_up_proj"]), up(d["down_proj"])
+        self.rb, self.b1, self.b2 = up(d["router_bias"]), up(d["b1"]), up(d["b2"])
+        self.dt = moe.BF16 if w.dtype == "bf16" else moe.F32
+        self.act = moe.ACT_NAMES[w.act]
+        self.ws = torch.empty(moe.workspace_size(w.T, w.D, w.F, w.E, w.K, self.dt, self.act),
+                              dtype=torch.uint8, device=dev)
+        self.out = torch.empty_like(self.x)
+        self.sel = torch.empty(w.T, w.K, dtype=torch.int64, device=dev)
+        self.wts = torch.empty(w.T, w.K, dtype=torch.float32, device=dev)
+        self.ext = ext_opts
+        self.stream = torch.cuda.current_stream(dev)
+
+    def step(self, xin=None, o=None, s=None):
+        from mixture_experts_ffn_09_b200 import moe
+        w = self.w
+        xin = self.x if xin is None else xin
+        o = self.out if o is None else o
+        s = self.stream if s is None else s
+        if self.ext:
+            moe.ffn_forward_ex(xin, self.router, self.gu, self.dn, w.E, w.K, w.norm_topk_prob,
+                               self.act, o, self.sel, self.wts, self.rb, self.b1, self.b2, None,
+                               self.ws, s, **self.ext)
+        else:
+            moe.ffn_forward(xin, self.router, self.gu, self.dn, w.E, w.K, w.norm_topk_prob,
+                            self.act, o, self.sel, self.wts, self.rb, self.b1, self.b2, None,
+                            self.ws, s)
+
+    def expert_load(self):
+        import numpy as np
+        return np.bincount(self.sel.cpu().numpy().ravel(), minlength=self.w.E)
+
+
+def time_steps(layer, steps, wd, world, local, what):
+    """Device time of `steps` forwards between CUDA events on the launching
+    stream, bracketed by a barrier and a synchronize; clocks sampled through
+    NVML meanwhile.  Returns (ms of this rank, launches, clocks)."""
+    import torch
+    from mixture_experts_ffn_09_b200 import moe
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    wd.sync(f"before {what}")
+    clocks = ClockSampler(local, pci_bus_id=cuda_pci_bus_id(local))
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    n_launch0 = moe.kernel_launches()
+    t0.record(layer.stream)
+    wd.run(steps, layer.step, what)
+    t1.record(layer.stream)
+    launches = moe.kernel_launches() - n_launch0
+    wd.sync(what)
+    clk = clocks.stop()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    return t0.elapsed_time(t1), launches, clk
+
+
+def stage_pass(layer, n, wd, local, what):
+    """Per-stage CUDA-event times of n forwards (events between the kernels
+    on the launching stream, so not the headline number), with the clocks
+    sampled through NVML during the pass.  Returns (ms per call by stage,
+    clocks)."""
+    from mixture_experts_ffn_09_b200 import moe
+    clocks = ClockSampler(local, pci_bus_id=cuda_pci_bus_id(local))
+    clocks.start()
+    moe.profile_enable(True)
+    wd.run(n, layer.step, what)
+    wd.sync(what)
+    stage_ms, calls = moe.profile_read()
+    moe.profile_enable(False)
+    clk = clocks.stop()
+    return {k: v / max(calls, 1) for k, v in stage_ms.items()}, clk
+
+
+def uses_pair_gemm(w, gemm: str) -> bool:
+    return w.dtype == "bf16" and (gemm == "2sm" or (gemm == "auto" and w.T * w.K >= 512 * w.E))
+
+
+def gate_up_roofline(w, per_call, touched, peaks, gemm, timed_s, stage_clk):
+    """Roofline of the dominant kernel, the gate_up grouped GEMM, from its
+    CUDA-event time: routed FLOPs against the bf16 tensor peak at large T,
+    the bytes it must move against the HBM copy bandwidth at small T."""
+    t_gu = per_call["gate_up"] / 1e3
+    pair = uses_pair_gemm(w, gemm)
+    if w.dtype != "bf16":
+        kname = "gemm_simt_f32_kernel<silu_gated> (gate_up, fp32 FMA)"
+    elif pair:
+        kname = "grouped_gemm_pair_kernel<silu_gated> (gate_up, CTA pairs)"
+    else:
+        kname = "grouped_gemm_tc_kernel<silu_gated> (gate_up, one CTA per tile)"
+    if w.T * w.K <= 512:
+        achieved = gate_up_bytes(w, touched) / t_gu / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "peak_source": peaks["source"] + " hbm copy",
+                "frac_of_nominal_8tbs": round(achieved / NOMINAL["hbm_gbs"], 4),
+                "algorithmic_bytes_per_launch": gate_up_bytes(w, touched)}
+    else:
+        fl = gate_up_flops(w)
+        achieved = fl / t_gu / 1e12
+        sustained = timed_s >= SUSTAINED_AFTER_S
+        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+        roof = {"kernel": kname, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": peaks["source"] + (
+                    " bf16 sustained (the timed loop lasted %.1f s)" % timed_s if sustained else
+                    " bf16 burst (the timed loop lasted %.2f s, too short to settle at the power cap)"
+                    % timed_s),
+                "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4),
+                "frac_of_sustained_peak": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                "frac_of_datasheet_2250": round(achieved / NOMINAL["bf16_tflops"], 4),
+                "algorithmic_flops_per_launch": fl}
+        mhz = stage_clk.get("sm_mhz")
+        if mhz:
+            per_clk = fl / (t_gu * mhz * 1e6)
+            roof["achieved_per_clock"] = {
+                "flop_per_clk": round(per_clk, 1), "sm_mhz": mhz,
+                "peak_flop_per_clk": SMS * PEAK_FLOP_PER_CLK_PER_SM,
+                "frac": round(per_clk / (SMS * PEAK_FLOP_PER_CLK_PER_SM), 4),
+                "how": "gate_up FLOP / (CUDA-event time x median SM clock of the per-stage pass); "
+                       "peak 148 SMs x 8192 dense bf16 FLOP per clock"}
+    roof["avg_launch_ms"] = round(per_call["gate_up"], 4)
+    return roof
+
+
+def measure_extra(w, args, dev, local, world, peaks):
+    """One more workload in the same process: its own inputs, warm-up,
+    timed forwards and per-stage pass.  The numbers every config is judged
+    on, without the end-to-end and CPU legs of the headline."""
+    from mixture_experts_ffn_09_b200 import moe, synth
+    d = synth.make_inputs(w)
+    layer = Layer(w, d, dev, args)
+    wd = Watchdog(dev, layer.stream, args.watchdog)
+    for i in range(max(args.warmup, 3)):
+        layer.step()
+        wd.sync(f"{w.name} warm-up step {i}")
+    st = moe.device_status(layer.stream)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"{w.name}: device status after warm-up: {moe.status_string(st)}")
+    load = layer.expert_load()
+    touched = int((load > 0).sum())
+    steps = max(5, min(args.steps, args.extra_steps))
+    local_ms, launches, clk = time_steps(layer, steps, wd, world, local, f"{w.name} timed region")
+    ms_step, tok_s = throughput(local_ms, steps, w.T, world, dev)
+    per_call, sclk = stage_pass(layer, max(5, min(steps, 50)), wd, local, f"{w.name} per-stage pass")
+    rflops = routed_flops(w)
+    abytes = algorithmic_bytes(w, touched)
+    r = {"config": workload_config(w, world), "steps": steps, "ms_per_step": round(ms_step, 4),
+         "tokens_per_s": round(tok_s, 1), "routed_tflops": round(world * rflops / (ms_step / 1e3) / 1e12, 3),
+         "stages_ms": {k: round(v, 4) for k, v in per_call.items()}, "gpu_launches": launches,
+         "experts_touched": touched, "clocks": clk}
+    if w.dtype == "bf16":
+        r["roofline"] = gate_up_roofline(w, per_call, touched, peaks, args.gemm, local_ms / 1e3, sclk)
+        if w.T * w.K <= 512:
+            # weight streaming: the whole step against the HBM copy bandwidth
+            r["step_hbm"] = {"algorithmic_bytes": abytes,
+                             "achieved_gbs": round(abytes / (ms_step / 1e3) / 1e9, 1),
+                             "frac_of_measured": round(abytes / (ms_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                             "frac_of_nominal_8tbs": round(abytes / (ms_step / 1e3) / 1e9 / NOMINAL["hbm_gbs"], 4)}
+        else:
+            r["step_tensor"] = {
+                "frac_of_burst_peak": round(rflops / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+                "frac_of_datasheet_2250": round(rflops / (ms_step / 1e3) / 1e12 / NOMINAL["bf16_tflops"], 4)}
+    else:
+        r["bound"] = "latency (a few small launches; inputs fit in L2)"
+    del layer
+    return r
+
+
 def run_ours(args, w):
     import numpy as np
     import torch
@@ -358,25 +563,6 @@ def run_ours(args, w):
     dev = torch.device("cuda", local)
     d = synth.make_inputs(w)
 
-    def up(a):
-        if a is None:
-            return None
-        if a.dtype == np.uint16:
-            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
-        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-
-    x, router, gu, dn = up(d["x"]), up(d["router"]), up(d["gate_up_proj"]), up(d["down_proj"])
-    rb, b1, b2 = up(d["router_bias"]), up(d["b1"]), up(d["b2"])
-    x = x.reshape(w.T, w.D)
-    dt = moe.BF16 if w.dtype == "bf16" else moe.F32
-    act = moe.ACT_NAMES[w.act]
-    ws = torch.empty(moe.workspace_size(w.T, w.D, w.F, w.E, w.K, dt, act), dtype=torch.uint8,
-                     device=dev)
-    out = torch.empty_like(x)
-    sel = torch.empty(w.T, w.K, dtype=torch.int64, device=dev)
-    wts = torch.empty(w.T, w.K, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
     ext = dict(score=args.score, dynamic_threshold=args.dynamic_threshold,
                capacity_factor=args.capacity_factor, seq_len=args.seq_len)
     if args.selection_bias > 0:
@@ -390,14 +576,9 @@ def run_ours(args, w):
         ext["slot_kept"] = kept
         if args.balance:
             ext["balance"] = bal
-
-    def step(xin=x, o=out, s=stream):
-        if use_ext:
-            moe.ffn_forward_ex(xin, router, gu, dn, w.E, w.K, w.norm_topk_prob, act, o, sel, wts,
-                               rb, b1, b2, None, ws, s, **ext)
-        else:
-            moe.ffn_forward(xin, router, gu, dn, w.E, w.K, w.norm_topk_prob, act, o, sel, wts, rb,
-                            b1, b2, None, ws, s)
+    layer = Layer(w, d, dev, args, ext if use_ext else None)
+    x, out, stream, dt = layer.x, layer.out, layer.stream, layer.dt
+    step = layer.step
 
     wd = Watchdog(dev, stream, args.watchdog)
     for i in range(max(args.warmup, 3)):
@@ -406,7 +587,7 @@ def run_ours(args, w):
     st = moe.device_status(stream)
     if st != moe.MOE_OK:
         raise RuntimeError(f"device status after warm-up: {moe.status_string(st)}")
-    load = np.bincount(sel.cpu().numpy().ravel(), minlength=w.E)
+    load = layer.expert_load()
     touched = int((load > 0).sum())
     ext_stats = {}
     if use_ext:
@@ -417,35 +598,14 @@ def run_ours(args, w):
                                             [round(float(v), 6) for v in bal.cpu().numpy()]))
 
     # ---------------- timed region: K forwards, device events on the stream
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    wd.sync("before the timed region")
-    clocks = ClockSampler(local, pci_bus_id=cuda_pci_bus_id(local))
-    clocks.start()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    n_launch0 = moe.kernel_launches()
-    t0.record(stream)
-    wd.run(args.steps, step, "timed region")
-    t1.record(stream)
-    timed_launches = moe.kernel_launches() - n_launch0
-    wd.sync("timed region")
-    clk = clocks.stop()
-    local_ms = t0.elapsed_time(t1)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    local_ms, timed_launches, clk = time_steps(layer, args.steps, wd, world, local, "timed region")
     ms_step, tokens_per_s = throughput(local_ms, args.steps, w.T, world, dev)
 
     # ---------------- per-stage times: a separate pass with CUDA events
     # around every kernel on the launching stream (the events sit between
-    # the kernels, so this pass is not the headline number)
-    moe.profile_enable(True)
-    wd.run(max(1, min(args.steps, 50)), step, "per-stage pass")
-    wd.sync("per-stage pass")
-    stage_ms, calls = moe.profile_read()
-    moe.profile_enable(False)
+    # the kernels, so this pass is not the headline number), clocks sampled
+    per_call, stage_clk = stage_pass(layer, max(20, min(args.steps, 50)), wd, local,
+                                     "per-stage pass")
     st = moe.device_status(stream)
     if st != moe.MOE_OK:
         raise RuntimeError(f"device status after timing: {moe.status_string(st)}")
@@ -455,8 +615,7 @@ def run_ours(args, w):
     # step i-1 computes, and step i's output is read back on another while
     # step i+1 computes (two device buffers each); every step still moves
     # its own input and output bytes inside the timed region.
-    xh = torch.from_numpy(np.ascontiguousarray(d["x"]).view(np.int16 if dt == moe.BF16 else np.float32))
-    xh = (xh.view(torch.bfloat16) if dt == moe.BF16 else xh).reshape(w.T, w.D).pin_memory()
+    xh = _readonly_view(d["x"]).reshape(w.T, w.D).pin_memory()
     oh = [torch.empty_like(xh).pin_memory() for _ in range(2)]
     xd = [torch.empty_like(x) for _ in range(2)]
     od = [torch.empty_like(out) for _ in range(2)]
@@ -509,32 +668,11 @@ def run_ours(args, w):
 
     # ---------------- roofline of the dominant kernel (gate_up)
     peaks = load_peaks()
-    per_call = {k: v / max(calls, 1) for k, v in stage_ms.items()}
     dom = max(per_call, key=per_call.get)
-    t_gu = per_call["gate_up"] / 1e3
-    hbm_bound = w.T * w.K <= 512
-    pair = args.gemm == "2sm" or (args.gemm == "auto" and w.T * w.K >= 512 * w.E)
-    kname = ("grouped_gemm_pair_kernel<silu_gated> (gate_up, CTA pairs)" if pair
-             else "grouped_gemm_tc_kernel<silu_gated> (gate_up, one CTA per tile)")
-    if hbm_bound:
-        achieved = gate_up_bytes(w, touched) / t_gu / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"kernel": kname, "bound": "hbm",
-                "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "peak_source": peaks["source"] + " hbm copy",
-                "algorithmic_bytes_per_launch": gate_up_bytes(w, touched)}
-    else:
-        achieved = gate_up_flops(w) / t_gu / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roof = {"kernel": kname, "bound": "tensor",
-                "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4),
-                "peak_source": peaks["source"] + " bf16 sustained (kernel timed inside a long loop)",
-                "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4),
-                "frac_of_datasheet_2250": round(achieved / NOMINAL["bf16_tflops"], 4),
-                "algorithmic_flops_per_launch": gate_up_flops(w)}
-    roof["traffic"] = stored_traffic(w.name, "gate_up_pair" if pair else "gate_up")
-    roof["avg_launch_ms"] = round(per_call["gate_up"], 4)
+    roof = gate_up_roofline(w, per_call, touched, peaks, args.gemm, local_ms / 1e3, stage_clk)
+    roof["traffic"] = stored_traffic(w.name, "gate_up_pair" if uses_pair_gemm(w, args.gemm)
+                                     else "gate_up")
+    roof["stage_pass_clocks"] = stage_clk
 
     rflops = routed_flops(w)
     abytes = algorithmic_bytes(w, touched)
@@ -583,6 +721,17 @@ def run_ours(args, w):
             result["cpu_baseline"]["single_core"] = {
                 "value": round(r1, 4), "unit": UNIT, "cores": 1,
                 "sample": f"{n1} tokens, BLAS held to one thread ({s1:.1f} s)"}
+
+    # ---------------- every other config, same process, after the headline
+    extra = [] if args.no_workloads else [synth.WORKLOADS[n] for n in EXTRA_WORKLOADS
+                                          if n != w.name]
+    if extra:
+        del layer, xd, od, xh, oh
+        torch.cuda.empty_cache()
+        result["workloads"] = {}
+        for ew in extra:
+            result["workloads"][ew.name] = measure_extra(ew, args, dev, local, world, peaks)
+            torch.cuda.empty_cache()
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -655,6 +804,10 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample (cpu_baseline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time only the selected workload (skip the other configs)")
+    ap.add_argument("--extra-steps", type=int, default=100,
+                    help="timed forwards of each other config (at most --steps)")
     ap.add_argument("--gemm", choices=["auto", "1sm", "2sm"], default="auto",
                     help="bf16 grouped GEMM: automatic, one CTA per tile, or CTA pairs")
     ap.add_argument("--score", choices=["softmax", "sigmoid"], default="softmax")
