@@ -28,6 +28,16 @@
 // matching 128 up rows, so accumulator columns [0,128) are gate and
 // [128,256) up in both CTAs, exactly as in the one-CTA kernel.
 //
+// Tiles are handed out dynamically, in order: the leader's producer takes
+// the next tile index from a global counter (zeroed each forward by the
+// scatter kernel) and publishes it through a small ring in shared memory to
+// the leader's MMA issuer and epilogue warps and, by a store into the peer's
+// shared memory and a remote barrier arrival, to the peer's producer and
+// epilogue warps.  Row blocks that share a weight tile are then taken within
+// a few tiles of each other wherever the pairs stand, so the weight tile is
+// read from DRAM once and served from L2 to the others; and pairs that draw
+// cheap tiles (swapped tails) simply take more of them.
+//
 // A pair tile covers 256 rows of one expert; rows past the expert's end are
 // computed and not stored.  The exception is an expert's last row block when
 // it holds at most `swap_max` rows (a short tail): that tile runs with the
@@ -62,6 +72,10 @@ constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int WB_BOX = 16;      // gate (then up) rows per group of the interleaved staging
 constexpr int kSwapMax = 128;   // longest tail that may run swapped (N = 128)
+constexpr int SCHED = 8;        // tile indices in flight from the scheduler to the roles
+// Readers of each published tile index, who release its slot: the leader's
+// MMA issuer and 4 epilogue warps, the peer's producer and 4 epilogue warps.
+constexpr int SCHED_READERS = 10;
 
 // Token-row views for swapped tails: box heights 8, 16, 32 and 64 rows.
 struct TokMaps {
@@ -83,6 +97,7 @@ struct Params {
   const float* bias;
   unsigned int* err;
   int swap_max;       // an expert's last block of at most this many rows runs swapped (0: never)
+  int* tile_counter;  // next tile to hand out; zero at launch
 };
 
 struct Tail {
@@ -91,6 +106,9 @@ struct Tail {
   uint64_t tfull[2];         // both: accumulator ready
   uint64_t tempty[2];        // leader: 8 epilogue warps released the accumulator
   uint64_t mma_done;
+  uint64_t sfull[SCHED];     // both: the slot holds the next tile index for this CTA
+  uint64_t sempty[SCHED];    // leader: every reader of the slot has taken it
+  int sched_tile[SCHED];     // tile index, -1 = no more tiles
   uint32_t tmem_base;
   int abort;
   int total_tiles;
@@ -116,6 +134,20 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
+}
+__device__ __forceinline__ void st_cluster_s32(uint32_t cluster_addr, int v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+// Reads the index of the i-th tile this CTA works on from the scheduler
+// ring and releases the slot on the leader (any role but the leader's
+// producer, which writes it).  -1: no more tiles, or the wait gave up.
+__device__ __forceinline__ int sched_take(Tail* st, int i, volatile int* abort, unsigned int* err,
+                                          unsigned int site) {
+  const int slot = i % SCHED;
+  if (!mbar_wait_cluster(&st->sfull[slot], (i / SCHED) & 1u, abort, err, site)) return -1;
+  const int t = st->sched_tile[slot];
+  mbar_arrive_cluster(map_to_rank(&st->sempty[slot], 0));
+  return t;
 }
 // TMA load into this CTA's shared memory whose completion is counted on the
 // barrier at `bar_cluster_addr` (the leader's, for a pair).
@@ -245,8 +277,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   const bool leader = rank == 0;
   const int E = p.E;
   const int n_tiles = (p.n_out + BN_OUT - 1) / BN_OUT;
-  const int cluster_id = blockIdx.x >> 1;
-  const int num_clusters = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -258,6 +288,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&st->tempty[a], 8);
     }
     mbar_init(&st->mma_done, 1);
+    for (int j = 0; j < SCHED; ++j) {
+      mbar_init(&st->sfull[j], 1);
+      mbar_init(&st->sempty[j], SCHED_READERS);
+    }
     st->abort = 0;
     mbar_fence_init();
   }
@@ -306,7 +340,28 @@ __global__ void __launch_bounds__(THREADS, 1)
     int stage = 0;
     uint32_t phase = 0, used = 0, last_parity = 0;
     const int rows_live = st->off[E];
-    for (int t = cluster_id; t < total; t += num_clusters) {
+    for (int i = 0;; ++i) {
+      // the next tile: the leader takes it from the counter and publishes it
+      // to both CTAs; the peer reads it from its own ring
+      int t = -1;
+      if (lane == 0) {
+        if (leader) {
+          const int slot = i % SCHED;
+          if (mbar_wait(&st->sempty[slot], ((i / SCHED) & 1u) ^ 1u, abort, p.err,
+                        SITE_PAIR_PRODUCER)) {
+            t = atomicAdd(p.tile_counter, 1);
+            if (t >= total) t = -1;
+          }
+          st->sched_tile[slot] = t;
+          st_cluster_s32(map_to_rank(&st->sched_tile[slot], 1), t);
+          mbar_arrive(&st->sfull[slot]);
+          mbar_arrive_cluster(map_to_rank(&st->sfull[slot], 1));
+        } else {
+          t = sched_take(st, i, abort, p.err, SITE_PAIR_PRODUCER);
+        }
+      }
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (t < 0) break;
       if (!__shfl_sync(0xffffffffu, lane == 0 ? static_cast<int>(!*abort) : 0, 0)) break;
       int e, m_blk, n_blk;
       decode_tile(st, E, n_tiles, t, e, m_blk, n_blk);
@@ -317,9 +372,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       int tok[4] = {0, 0, 0, 0};
       if (GATHER) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = rowA + 4 * lane + i;
-          tok[i] = r < rows_live ? __ldg(p.perm + r) / p.K : 0;
+        for (int q = 0; q < 4; ++q) {
+          const int r = rowA + 4 * lane + q;
+          tok[q] = r < rows_live ? __ldg(p.perm + r) / p.K : 0;
         }
       }
       bool ok = true;
@@ -396,8 +451,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(BMP, BN_MMA);
       int stage = 0;
       uint32_t phase = 0;
-      int i = 0;
-      for (int t = cluster_id; t < total; t += num_clusters, ++i) {
+      for (int i = 0;; ++i) {
+        const int t = sched_take(st, i, abort, p.err, SITE_PAIR_MMA);
+        if (t < 0) break;
         const int acc = i & 1;
         const uint32_t aph = (i >> 1) & 1;
         if (!mbar_wait(&st->tempty[acc], aph ^ 1u, abort, p.err, SITE_PAIR_MMA)) break;
@@ -451,8 +507,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int lane_base = (warp & 3) * 32;
     const uint32_t tempty_leader0 = map_to_rank(&st->tempty[0], 0);
     const uint32_t tempty_leader1 = map_to_rank(&st->tempty[1], 0);
-    int i = 0;
-    for (int t = cluster_id; t < total; t += num_clusters, ++i) {
+    for (int i = 0;; ++i) {
+      int t = lane == 0 ? sched_take(st, i, abort, p.err, SITE_PAIR_EPILOGUE) : -1;
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (t < 0) break;
       int e, m_blk, n_blk;
       decode_tile(st, E, n_tiles, t, e, m_blk, n_blk);
       const int acc = i & 1;
@@ -684,13 +742,13 @@ cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
 
 cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* W,
                                 const int* offsets, int E, int Kdim, int N, int w_rows_per_expert,
-                                const float* bias, void* C, unsigned int* err, cudaStream_t s,
-                                const int* gather_perm, int gather_K, int gather_rows,
-                                int swap_max) {
+                                const float* bias, void* C, unsigned int* err, int* tile_counter,
+                                cudaStream_t s, const int* gather_perm, int gather_K,
+                                int gather_rows, int swap_max) {
   CUtensorMap ma, mb, mgu;
   TokMaps tok;
   const bool gather = gather_perm != nullptr;
-  if (swap_max < 0 || swap_max > kSwapMax) return cudaErrorInvalidValue;
+  if (swap_max < 0 || swap_max > kSwapMax || !tile_counter) return cudaErrorInvalidValue;
   if (!make_map(&ma, A, static_cast<uint64_t>(gather ? gather_rows : a_rows),
                 static_cast<uint64_t>(Kdim), gather ? 1u : 128u) ||
       !make_map(&mb, W, static_cast<uint64_t>(E) * w_rows_per_expert, static_cast<uint64_t>(Kdim)))
@@ -719,6 +777,7 @@ cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* 
   p.bias = bias;
   p.err = err;
   p.swap_max = swap_max;
+  p.tile_counter = tile_counter;
   const int bn_out = (act == kSiluGated) ? 128 : 256;
   const long long tiles_bound =
       (static_cast<long long>(a_rows) / BMP + E) * ((N + bn_out - 1) / bn_out);

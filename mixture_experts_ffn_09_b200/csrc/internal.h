@@ -12,6 +12,12 @@ namespace moe {
 constexpr int kMaxExperts = 256;
 constexpr int kRouterTokensPerCta = 32;   // tokens per router CTA = per permute block
 constexpr int kTileM = 128;               // rows of one grouped-GEMM tile
+// Tile counters of the grouped GEMMs' dynamic schedulers, one per GEMM of a
+// forward, each on its own 128-byte line: kSchedInts ints in the workspace,
+// zeroed by the scatter kernel of the same forward.
+constexpr int kSchedInts = 64;
+constexpr int kSchedGateUp = 0;
+constexpr int kSchedDown = 32;
 
 enum DType : int { kF32 = 0, kBF16 = 1 };
 
@@ -66,9 +72,11 @@ cudaError_t launch_permute_scan(const int* blockcounts, int B, int E, int* block
 // Slots whose in-block rank reaches the (clamped) block count, and slots
 // with the sentinel expert, get no row: pos = -1, slot_kept = 0.
 // blockbase / totals null: the kernel scans the block counts itself.
+// sched (kSchedInts, or null): block 0 zeroes the GEMMs' tile counters.
 cudaError_t launch_permute_scatter(const int* idx32, const int* blockbase, const int* totals,
                                    const int* blockcounts, int T, int K, int E, int* offsets,
-                                   int* perm, int* pos, uint8_t* slot_kept, cudaStream_t s);
+                                   int* perm, int* pos, uint8_t* slot_kept, int* sched,
+                                   cudaStream_t s);
 
 // x_perm[pos[t, k], :] = x[t, :] for every slot that was given a row
 // (pos >= 0; perm is the inverse map, offsets[E] the live row count): by
@@ -103,12 +111,14 @@ cudaError_t launch_gemm_tc(int act, const void* A, int a_rows, const void* W, co
 
 // Same GEMM on CTA pairs (tcgen05 cta_group::2, 256-row tiles).  An expert's
 // last row block of at most swap_max rows (0..255; 0: never) runs as a
-// swapped-operand tile whose N is the block's rows rounded up to 16.
+// swapped-operand tile whose N is the block's rows rounded up to 16.  The
+// persistent pairs take tiles in order from *tile_counter, which must be
+// zero when the kernel starts (the scatter kernel zeroes it each forward).
 cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* W,
                                 const int* offsets, int E, int Kdim, int N, int w_rows_per_expert,
-                                const float* bias, void* C, unsigned int* err, cudaStream_t s,
-                                const int* gather_perm = nullptr, int gather_K = 0,
-                                int gather_rows = 0, int swap_max = 0);
+                                const float* bias, void* C, unsigned int* err, int* tile_counter,
+                                cudaStream_t s, const int* gather_perm = nullptr,
+                                int gather_K = 0, int gather_rows = 0, int swap_max = 0);
 
 int num_sms();
 unsigned long long kernel_launches();   // accepted launches so far (note_launch)

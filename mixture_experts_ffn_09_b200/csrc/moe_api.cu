@@ -41,13 +41,13 @@ constexpr long long kScatterScansItself = 4096;
 cudaError_t launch_gemm_bf16(int act, const void* A, int a_rows, const void* W,
                              const int* offsets, int E, int T, int K, int Kdim, int N,
                              int w_rows, const float* bias, void* C, unsigned int* err,
-                             cudaStream_t s, const int* gather_perm = nullptr) {
+                             int* tile_counter, cudaStream_t s, const int* gather_perm = nullptr) {
   const int mode = g_gemm_mode.load();
   const bool pair = mode == MOE_GEMM_2SM ||
                     (mode == MOE_GEMM_AUTO && static_cast<long long>(T) * K >= 512LL * E);
   if (pair)
-    return moe::launch_gemm_tc_pair(act, A, a_rows, W, offsets, E, Kdim, N, w_rows, bias, C, err, s,
-                                    gather_perm, K, T, g_tail_swap.load());
+    return moe::launch_gemm_tc_pair(act, A, a_rows, W, offsets, E, Kdim, N, w_rows, bias, C, err,
+                                    tile_counter, s, gather_perm, K, T, g_tail_swap.load());
   return moe::launch_gemm_tc(act, A, a_rows, W, offsets, E, static_cast<long long>(T) * K, Kdim, N,
                              w_rows, bias, C, err, s, gather_perm, K, T);
 }
@@ -236,7 +236,7 @@ struct StageTimer {
 
 // ------------------------------------------------------ workspace layout
 struct Layout {
-  size_t idx32, w32, bcount, bbase, totals, offsets, perm, pos, bal, xperm, h, y, total;
+  size_t idx32, w32, bcount, bbase, totals, offsets, sched, perm, pos, bal, xperm, h, y, total;
   int B, Rpad;
 };
 
@@ -257,6 +257,7 @@ Layout layout(int64_t T, int64_t D, int64_t F, int E, int K, int elem) {
   L.bbase = take(sizeof(int) * static_cast<size_t>(L.B) * E);
   L.totals = take(sizeof(int) * E);
   L.offsets = take(sizeof(int) * (E + 1));
+  L.sched = take(sizeof(int) * moe::kSchedInts);
   L.perm = take(sizeof(int) * R);
   L.pos = take(sizeof(int) * R);
   {
@@ -491,6 +492,7 @@ moe_status_t ffn_forward_impl(const void* x, const void* router, const void* gat
   int* bbase = reinterpret_cast<int*>(ws + L.bbase);
   int* totals = reinterpret_cast<int*>(ws + L.totals);
   int* offsets = reinterpret_cast<int*>(ws + L.offsets);
+  int* sched = reinterpret_cast<int*>(ws + L.sched);
   int* perm = reinterpret_cast<int*>(ws + L.perm);
   int* pos = reinterpret_cast<int*>(ws + L.pos);
   void* xperm = ws + L.xperm;
@@ -551,7 +553,7 @@ moe_status_t ffn_forward_impl(const void* x, const void* router, const void* gat
       if (!debug_wait(dev, s, "permute scan")) return cudaErrorTimeout;
     }
     r = moe::launch_permute_scatter(idx32, own_scan ? nullptr : bbase, own_scan ? nullptr : totals,
-                                    bcount, Ti, K, E, offsets, perm, pos, slot_kept, s);
+                                    bcount, Ti, K, E, offsets, perm, pos, slot_kept, sched, s);
     if (r != cudaSuccess) return r;
     if (!debug_wait(dev, s, "permute scatter")) return cudaErrorTimeout;
     if (fused_gather) return r;
@@ -564,14 +566,14 @@ moe_status_t ffn_forward_impl(const void* x, const void* router, const void* gat
   if (dt == MOE_BF16) {
     e = timer.run(2, [&] {
       return launch_gemm_bf16(gu_act, fused_gather ? x : xperm, L.Rpad, gate_up_proj, offsets, E,
-                              Ti, K, Di, Fi, gu_rows, b1, H, dev->err, s,
+                              Ti, K, Di, Fi, gu_rows, b1, H, dev->err, sched + moe::kSchedGateUp, s,
                               fused_gather ? perm : nullptr);
     });
     if (e != cudaSuccess) return cuda_fail(e, "gate_up launch");
     if (!debug_wait(dev, s, "gate_up GEMM")) return MOE_ERR_TIMEOUT;
     e = timer.run(3, [&] {
       return launch_gemm_bf16(2, H, L.Rpad, down_proj, offsets, E, Ti, K, Fi, Di, Di, b2, Y,
-                              dev->err, s);
+                              dev->err, sched + moe::kSchedDown, s);
     });
     if (e != cudaSuccess) return cuda_fail(e, "down launch");
     if (!debug_wait(dev, s, "down GEMM")) return MOE_ERR_TIMEOUT;

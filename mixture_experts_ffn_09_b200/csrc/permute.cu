@@ -72,7 +72,8 @@ constexpr int kScatterWarps = kScatterThreads / 32;
 __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
     const int* __restrict__ idx32, const int* __restrict__ blockbase, const int* __restrict__ totals,
     const int* __restrict__ blockcounts, int T, int K, int E, int* __restrict__ offsets,
-    int* __restrict__ perm, int* __restrict__ pos, uint8_t* __restrict__ slot_kept) {
+    int* __restrict__ perm, int* __restrict__ pos, uint8_t* __restrict__ slot_kept,
+    int* __restrict__ sched) {
   __shared__ int off[kMaxExperts + 1];
   __shared__ int base[kMaxExperts];
   __shared__ int kept[kMaxExperts];
@@ -115,8 +116,12 @@ __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
     off[E] = acc;
   }
   __syncthreads();
-  if (b == 0)
+  if (b == 0) {
     for (int e = threadIdx.x; e <= E; e += kScatterThreads) offsets[e] = off[e];
+    // the grouped GEMMs' tile counters start this forward at zero
+    if (sched)
+      for (int i = threadIdx.x; i < kSchedInts; i += kScatterThreads) sched[i] = 0;
+  }
   for (int e = threadIdx.x; e < E; e += kScatterThreads) {
     base[e] = off[e] + (blockbase ? blockbase[static_cast<size_t>(b) * E + e] : base[e]);
     kept[e] = blockcounts[static_cast<size_t>(b) * E + e];
@@ -269,10 +274,12 @@ cudaError_t launch_permute_scan(const int* blockcounts, int B, int E, int* block
 
 cudaError_t launch_permute_scatter(const int* idx32, const int* blockbase, const int* totals,
                                    const int* blockcounts, int T, int K, int E, int* offsets,
-                                   int* perm, int* pos, uint8_t* slot_kept, cudaStream_t s) {
+                                   int* perm, int* pos, uint8_t* slot_kept, int* sched,
+                                   cudaStream_t s) {
   const int B = (T + kRouterTokensPerCta - 1) / kRouterTokensPerCta;
   return launch_k(permute_scatter_kernel, dim3(B), dim3(kScatterThreads), 0, s, pdl_enabled(), 1,
-                  idx32, blockbase, totals, blockcounts, T, K, E, offsets, perm, pos, slot_kept);
+                  idx32, blockbase, totals, blockcounts, T, K, E, offsets, perm, pos, slot_kept,
+                  sched);
 }
 
 cudaError_t launch_gather_rows(const int* perm, const int* offsets, const int* pos, int T, int E,
