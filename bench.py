@@ -451,10 +451,33 @@ def uses_pair_gemm(w, gemm: str) -> bool:
     return w.dtype == "bf16" and (gemm == "2sm" or (gemm == "auto" and w.T * w.K >= 512 * w.E))
 
 
+FP32_LANES_PER_SM = 128             # fp32 FMA units per SM (4 sub-partitions x 32)
+
+
+def alu_roofline(w, per_call, stage_clk):
+    """Float32 layers run on CUDA cores: the dominant kernel (the one-kernel
+    small layer, else the fp32 gate_up GEMM) against the fp32 FMA rate,
+    148 SMs x 128 lanes x 2 FLOP per clock at the maximum SM clock."""
+    small = per_call.get("small_layer", 0.0) > 0
+    ms = per_call["small_layer"] if small else per_call["gate_up"]
+    fl = w.routed_flops() if small else gate_up_flops(w)
+    mhz = stage_clk.get("sm_max_mhz") or 1965
+    peak = SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+    achieved = fl / (ms / 1e3) / 1e12
+    return {"kernel": "small_layer_f32_kernel (the whole layer, one cluster)" if small
+            else "gemm_simt_f32_kernel<silu_gated> (gate_up, fp32 FMA)",
+            "bound": "alu", "achieved": round(achieved, 4), "peak": round(peak, 2),
+            "unit": "TFLOP/s", "frac": round(achieved / peak, 5),
+            "peak_source": f"derived: {SMS} SMs x {FP32_LANES_PER_SM} fp32 lanes x 2 FLOP x {mhz} MHz",
+            "algorithmic_flops_per_launch": fl, "avg_launch_ms": round(ms, 4)}
+
+
 def gate_up_roofline(w, per_call, touched, peaks, gemm, timed_s, stage_clk):
     """Roofline of the dominant kernel, the gate_up grouped GEMM, from its
     CUDA-event time: routed FLOPs against the bf16 tensor peak at large T,
     the bytes it must move against the HBM copy bandwidth at small T."""
+    if w.dtype != "bf16":
+        return alu_roofline(w, per_call, stage_clk)
     t_gu = per_call["gate_up"] / 1e3
     pair = uses_pair_gemm(w, gemm)
     if w.dtype != "bf16":
@@ -538,7 +561,8 @@ def measure_extra(w, args, dev, local, world, peaks):
                 "frac_of_burst_peak": round(rflops / (ms_step / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
                 "frac_of_datasheet_2250": round(rflops / (ms_step / 1e3) / 1e12 / NOMINAL["bf16_tflops"], 4)}
     else:
-        r["bound"] = "latency (a few small launches; inputs fit in L2)"
+        r["roofline"] = alu_roofline(w, per_call, sclk)
+        r["bound"] = "latency (one small launch; inputs fit in L2)"
     del layer
     return r
 
@@ -670,8 +694,8 @@ def run_ours(args, w):
     peaks = load_peaks()
     dom = max(per_call, key=per_call.get)
     roof = gate_up_roofline(w, per_call, touched, peaks, args.gemm, local_ms / 1e3, stage_clk)
-    roof["traffic"] = stored_traffic(w.name, "gate_up_pair" if uses_pair_gemm(w, args.gemm)
-                                     else "gate_up")
+    roof["traffic"] = (stored_traffic(w.name, "gate_up_pair" if uses_pair_gemm(w, args.gemm)
+                                      else "gate_up") if w.dtype == "bf16" else None)
     roof["stage_pass_clocks"] = stage_clk
 
     rflops = routed_flops(w)

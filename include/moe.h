@@ -351,7 +351,8 @@ MOE_API moe_status_t moe_device_error_peek(unsigned int* word);
 
 /* Number of kernels this library has launched in the process so far (all
    devices, all entry points; launches the CUDA runtime accepted).  A forward
-   launches 6 to 9 kernels depending on its size and options. */
+   launches 6 to 9 kernels depending on its size and options, or one for a
+   small float32 layer (E <= 8, T*K <= 256, no routing options). */
 MOE_API unsigned long long moe_kernel_launches(void);
 
 /* Comma-separated names of the sites set in an error word (static storage
@@ -371,11 +372,13 @@ MOE_API moe_status_t moe_debug_bounded_wait(int timeout_ms, void* stream);
 /*
  * Stage profiler.  While enabled, moe_ffn_forward records CUDA events
  * around each of its kernels on the caller's stream (router, permute,
- * gate_up, down, combine).  moe_profile_read synchronises on the recorded
- * events, adds their durations (milliseconds) into ms[0..n_stages) and
- * returns the number of forward calls covered, then resets the counters.
+ * gate_up, down, combine; a small float32 layer that runs as one kernel
+ * records it as small_layer).  moe_profile_read synchronises on the
+ * recorded events, adds their durations (milliseconds) into
+ * ms[0..n_stages) and returns the number of forward calls covered, then
+ * resets the counters.
  */
-#define MOE_NUM_STAGES 5
+#define MOE_NUM_STAGES 6
 MOE_API moe_status_t moe_profile_enable(int enable);
 MOE_API int moe_profile_read(float* ms, int n_stages);
 MOE_API const char* moe_stage_name(int stage);

@@ -315,6 +315,12 @@ moe_status_t check_opts(const moe_route_opts_t* o, bool forward) {
   return MOE_OK;
 }
 
+// True when any routing option differs from its default (off).
+bool opts_active(const moe_route_opts_t* o) {
+  return o && (o->score != MOE_SCORE_SOFTMAX || o->selection_bias || o->dynamic_threshold > 0.f ||
+               o->capacity_factor > 0.f || o->slot_kept || o->balance);
+}
+
 void apply_opts(moe::RouteArgs& a, const moe_route_opts_t* o) {
   if (!o) return;
   a.score = o->score == MOE_SCORE_SIGMOID ? 1 : 0;
@@ -362,7 +368,8 @@ const char* moe_status_string(moe_status_t s) {
 }
 
 const char* moe_stage_name(int stage) {
-  static const char* names[MOE_NUM_STAGES] = {"router", "permute", "gate_up", "down", "combine"};
+  static const char* names[MOE_NUM_STAGES] = {"router", "permute", "gate_up", "down", "combine",
+                                              "small_layer"};
   return (stage >= 0 && stage < MOE_NUM_STAGES) ? names[stage] : "";
 }
 
@@ -511,7 +518,21 @@ moe_status_t ffn_forward_impl(const void* x, const void* router, const void* gat
   const int gu_rows = act == MOE_ACT_SILU_GATED ? 2 * Fi : Fi;
 
   StageTimer timer(s);
-  cudaError_t e = timer.run(0, [&] {
+  cudaError_t e;
+  if (dt == MOE_F32 && !opts_active(opts) && moe::small_layer_fits(Ti, Di, Fi, E, K, gu_act == 0)) {
+    // a small float32 layer: the whole forward in one launch
+    e = timer.run(5, [&] {
+      return moe::launch_small_layer_f32(
+          static_cast<const float*>(x), static_cast<const float*>(router), router_bias,
+          static_cast<const float*>(gate_up_proj), static_cast<const float*>(down_proj), b1, b2,
+          Ti, Di, Fi, E, K, norm_topk_prob ? 1 : 0, gu_act == 0 ? 1 : 0, static_cast<float*>(out),
+          selected_experts, routing_weights, router_logits, s);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "small-layer launch");
+    if (!debug_wait(dev, s, "small layer")) return MOE_ERR_TIMEOUT;
+    return MOE_OK;
+  }
+  e = timer.run(0, [&] {
     moe::RouteArgs a{};
     a.x = x;
     a.router = router;

@@ -43,7 +43,7 @@ ACT_NAMES = {"silu_gated": ACT_SILU_GATED, "silu": ACT_SILU_GATED, "relu": ACT_R
 F32 = 0
 BF16 = 1
 F64 = 2
-NUM_STAGES = 5
+NUM_STAGES = 6
 
 SCORE_SOFTMAX = 0
 SCORE_SIGMOID = 1

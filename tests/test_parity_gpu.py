@@ -482,6 +482,54 @@ def test_kernel_launch_count_per_forward():
     assert launches(256, 8, capacity_factor=1.0, balance=bal) == 8
 
 
+@pytest.mark.parametrize("name", [synth.DENSE_RELU.name, synth.SILU_SMALL.name, "random"])
+def test_small_float32_layer_runs_as_one_kernel(name):
+    """A small float32 layer (E <= 8, T*K <= 256, no routing options) runs
+    as one clustered kernel; asking for slot_kept sends the same layer down
+    the general six-kernel path.  Both match the oracle, and each other."""
+    import torch
+    from mixture_experts_ffn_09_b200 import moe
+    if name == "random":
+        d, E, K, act = synth.random_case(91, 37, 24, 40, 5, dtype="f32", weight_std=0.3), 5, 3, "silu_gated"
+    else:
+        w = synth.WORKLOADS[name]
+        d, E, K, act = synth.make_inputs(w), w.E, w.K, w.act
+    h = PL.host_views(d)
+    dev = PL.to_device(d)
+    x = dev["x"].reshape(-1, dev["x"].shape[-1])
+    T, D = x.shape
+    F = dev["down_proj"].shape[-1]
+    a = moe.ACT_NAMES[act]
+    ws = torch.empty(moe.workspace_size(T, D, F, E, K, moe.F32, a), dtype=torch.uint8, device="cuda")
+    res = []
+    for general in (False, True):
+        out = torch.empty_like(x)
+        sel = torch.empty(T, K, dtype=torch.int64, device="cuda")
+        wt = torch.empty(T, K, dtype=torch.float32, device="cuda")
+        kept = torch.empty(T, K, dtype=torch.uint8, device="cuda")
+        n0 = moe.kernel_launches()
+        moe.ffn_forward_ex(x, dev["router"], dev["gate_up_proj"], dev["down_proj"], E, K, True, a,
+                           out, sel, wt, dev["router_bias"], dev["b1"], dev["b2"], None, ws,
+                           **({"slot_kept": kept} if general else {}))
+        n = moe.kernel_launches() - n0
+        assert moe.device_status() == moe.MOE_OK
+        assert n == (6 if general else 1)
+        res.append({"out": out.cpu().numpy().astype(np.float64), "sel": sel.cpu().numpy(),
+                    "w": wt.cpu().numpy().astype(np.float64)})
+    r = O.moe_route(h["x"].reshape(T, D), h["router"], K, True, h["router_bias"])
+    for g in res:
+        clear = PL.check_routing(g, r, K, True)
+        ref = O.moe_ffn_forward(h["x"].reshape(T, D), h["router"], h["gate_up_proj"], h["down_proj"],
+                                K, True, act, h["router_bias"], h["b1"], h["b2"])["out"]
+        if (~clear).any():
+            un = np.nonzero(~clear)[0]
+            ref[un] = PL.oracle_out_for(h, un, g["sel"][un], K, True, act)
+        PL.check_out(g["out"], ref, "f32")
+    same = (res[0]["sel"] == res[1]["sel"]).all(1)
+    assert same.mean() > 0.95
+    PL.check_out(res[0]["out"][same], res[1]["out"][same], "f32", "one kernel vs six")
+
+
 def _random_shapes(n, seed):
     """Seeded layer shapes across the supported ranges: bf16 needs D and F
     multiples of 8, any sizes on float32."""
