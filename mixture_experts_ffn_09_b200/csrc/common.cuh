@@ -195,6 +195,13 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   }
 }
 
+// silu(g) = g * sigmoid(g) = g / (1 + e^-g) for the bf16 epilogues: fast
+// exponential and division (a few ulp in fp32, far below the one rounding to
+// bf16 that follows).  Large negative g gives e^-g = inf and a result of -0.
+__device__ __forceinline__ float silu_bf16_epilogue(float g) {
+  return __fdividef(g, 1.f + __expf(-g));
+}
+
 // ------------------------------------------------------------------ TMA
 // 2-D tiled load of one box into shared memory, completing on `bar`.
 // c0 is the innermost (contiguous) coordinate in elements, c1 the row.

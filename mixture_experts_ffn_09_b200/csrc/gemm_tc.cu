@@ -320,8 +320,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int j = 0; j < 16; ++j) {
               const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
               const float u0 = __uint_as_float(u[2 * j]), u1 = __uint_as_float(u[2 * j + 1]);
-              const float h0 = g0 / (1.f + __expf(-g0)) * u0;
-              const float h1 = g1 / (1.f + __expf(-g1)) * u1;
+              const float h0 = silu_bf16_epilogue(g0) * u0;
+              const float h1 = silu_bf16_epilogue(g1) * u1;
               w[j] = pack_bf16x2(h0, h1);
             }
             store_row32(rowp, col0, p.n_out, w);

@@ -28,6 +28,16 @@
 // matching 128 up rows, so accumulator columns [0,128) are gate and
 // [128,256) up in both CTAs, exactly as in the one-CTA kernel.
 //
+// The last wave is split: when fewer tiles are left than pairs, the last
+// `pairs` tiles each run as two work items over the two halves of the
+// k-blocks.  The first half stores its fp32 accumulator to a scratch area
+// and sets one flag per epilogue warp; the second half waits (bounded) for
+// the flag of its warp and adds the stored partial before its own epilogue.
+// The two halves are consecutive items, so the first is always handed out
+// before the second, and the sum is always (second half) + (first half):
+// deterministic.  Pairs that would have idled through a mostly empty last
+// wave take half tiles instead.
+//
 // Tiles are handed out dynamically, in order: the leader's producer takes
 // the next tile index from a global counter (zeroed each forward by the
 // scatter kernel) and publishes it through a small ring in shared memory to
@@ -98,7 +108,48 @@ struct Params {
   unsigned int* err;
   int swap_max;       // an expert's last block of at most this many rows runs swapped (0: never)
   int* tile_counter;  // next tile to hand out; zero at launch
+  float* split_partial;   // first halves' fp32 accumulators (split last wave), or null
+  int* split_flags;       // one per split unit, CTA and epilogue warp; zero at launch
+  int split_cap;          // split units the scratch holds
 };
+
+// One scheduled work item: tile t over k-blocks [kb0, kb1); half -1 for a
+// whole tile, else 0 / 1 for the halves of split unit `slot`.
+struct Item {
+  int t, kb0, kb1, half, slot;
+};
+
+// The first `total - S` items are whole tiles; the last S tiles follow as
+// pairs of half items.
+__device__ __forceinline__ Item decode_item(int w, int total, int S, int num_kb) {
+  Item it;
+  const int first = total - S;
+  if (w < first) {
+    it.t = w;
+    it.kb0 = 0;
+    it.kb1 = num_kb;
+    it.half = -1;
+    it.slot = 0;
+    return it;
+  }
+  const int j = w - first;
+  const int mid = num_kb / 2;
+  it.t = first + (j >> 1);
+  it.half = j & 1;
+  it.slot = j >> 1;
+  it.kb0 = it.half ? mid : 0;
+  it.kb1 = it.half ? num_kb : mid;
+  return it;
+}
+
+__device__ __forceinline__ void flag_release(int* f) {
+  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(f), "r"(1) : "memory");
+}
+__device__ __forceinline__ int flag_acquire(const int* f) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+  return v;
+}
 
 struct Tail {
   uint64_t full[STAGES];     // leader: both CTAs' loads of a stage
@@ -331,6 +382,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = st->tmem_base;
   const int total = st->total_tiles;
   volatile int* abort = &st->abort;
+  // the last min(pairs, tiles) tiles run as k-halves when scratch is given
+  const int n_pairs = static_cast<int>(gridDim.x >> 1);
+  const int S = (p.split_partial && p.num_kb >= 2)
+                    ? min(min(n_pairs, total), p.split_cap)
+                    : 0;
+  const int total_items = total + S;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -350,7 +407,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (mbar_wait(&st->sempty[slot], ((i / SCHED) & 1u) ^ 1u, abort, p.err,
                         SITE_PAIR_PRODUCER)) {
             t = atomicAdd(p.tile_counter, 1);
-            if (t >= total) t = -1;
+            if (t >= total_items) t = -1;
           }
           st->sched_tile[slot] = t;
           st_cluster_s32(map_to_rank(&st->sched_tile[slot], 1), t);
@@ -363,8 +420,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       t = __shfl_sync(0xffffffffu, t, 0);
       if (t < 0) break;
       if (!__shfl_sync(0xffffffffu, lane == 0 ? static_cast<int>(!*abort) : 0, 0)) break;
+      const Item it = decode_item(t, total, S, p.num_kb);
       int e, m_blk, n_blk;
-      decode_tile(st, E, n_tiles, t, e, m_blk, n_blk);
+      decode_tile(st, E, n_tiles, it.t, e, m_blk, n_blk);
       const int rowA = st->off[e] + m_blk * BMP + static_cast<int>(rank) * BMC;
       const int rowB = (EPI == kSiluGated)
                            ? e * p.b_rows + n_blk * 128 + (leader ? 0 : p.up_off)
@@ -388,7 +446,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // gated: the first 16-row group of this CTA's 64 features, counted in
         // the weights' 16-row groups (the gated swap requires F % 16 == 0)
         const int g0 = (e * p.b_rows + n_blk * 128 + static_cast<int>(rank) * 64) / WB_BOX;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = it.kb0; kb < it.kb1; ++kb) {
           int good = 1;
           if (lane == 0) {
             good = mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err, SITE_PAIR_PRODUCER) ? 1 : 0;
@@ -412,7 +470,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!ok) break;
         continue;
       }
-      for (int kb = 0; kb < p.num_kb; ++kb) {
+      for (int kb = it.kb0; kb < it.kb1; ++kb) {
         int good = 1;
         if (lane == 0) {
           good = mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err, SITE_PAIR_PRODUCER) ? 1 : 0;
@@ -461,15 +519,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t d = tmem + acc * BN_MMA;
         bool ok = true;
         int sw = 0;
+        const Item it = decode_item(t, total, S, p.num_kb);
         if (!GATHER && p.swap_max > 0) {
           int e, m_blk, n_blk;
-          decode_tile(st, E, n_tiles, t, e, m_blk, n_blk);
+          decode_tile(st, E, n_tiles, it.t, e, m_blk, n_blk);
           sw = swap_rows(st, p.swap_max, e, m_blk);
         }
         if (sw) {
           // swapped tail: A = the weight rows (B slot), B = the token rows (A slot)
           const uint32_t idesc_sw = idesc_bf16_f32(BMP, 16 << swap_idx(sw));
-          for (int kb = 0; kb < p.num_kb; ++kb) {
+          for (int kb = it.kb0; kb < it.kb1; ++kb) {
             if (!mbar_wait(&st->full[stage], phase, abort, p.err, SITE_PAIR_MMA)) { ok = false; break; }
             tc_fence_after();
             const uint32_t w0 = smem_u32(sB + stage * B_BYTES);
@@ -477,12 +536,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k)
               umma_bf16_pair(d, sw128_kmajor_desc(w0 + k * 32), sw128_kmajor_desc(x0 + k * 32),
-                             idesc_sw, (kb | k) != 0 ? 1u : 0u);
+                             idesc_sw, (kb != it.kb0 || k != 0) ? 1u : 0u);
             umma_commit_pair(&st->empty[stage]);
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
           }
         } else {
-          for (int kb = 0; kb < p.num_kb; ++kb) {
+          for (int kb = it.kb0; kb < it.kb1; ++kb) {
             if (!mbar_wait(&st->full[stage], phase, abort, p.err, SITE_PAIR_MMA)) { ok = false; break; }
             tc_fence_after();
             const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
@@ -490,7 +549,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k)
               umma_bf16_pair(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
-                             (kb | k) != 0 ? 1u : 0u);
+                             (kb != it.kb0 || k != 0) ? 1u : 0u);
             umma_commit_pair(&st->empty[stage]);
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
           }
@@ -511,8 +570,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       int t = lane == 0 ? sched_take(st, i, abort, p.err, SITE_PAIR_EPILOGUE) : -1;
       t = __shfl_sync(0xffffffffu, t, 0);
       if (t < 0) break;
+      const Item it = decode_item(t, total, S, p.num_kb);
       int e, m_blk, n_blk;
-      decode_tile(st, E, n_tiles, t, e, m_blk, n_blk);
+      decode_tile(st, E, n_tiles, it.t, e, m_blk, n_blk);
       const int acc = i & 1;
       const uint32_t aph = (i >> 1) & 1;
       // every lane must agree before the warp-collective TMEM loads
@@ -520,6 +580,59 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tb = tmem + (static_cast<uint32_t>(lane_base) << 16) + acc * BN_MMA;
+      // split last wave: this warp's slice of the unit's partial accumulator,
+      // column-major over its 128 rows (column c of row r at c * 128 + r)
+      const int prow = lane_base + lane;
+      float* part = it.half >= 0
+                        ? p.split_partial + (static_cast<size_t>(it.slot) * 2 + rank) * (256 * 128)
+                        : nullptr;
+      int* flag = it.half >= 0 ? p.split_flags + (it.slot * 2 + static_cast<int>(rank)) * 4 + (warp & 3)
+                               : nullptr;
+      if (it.half == 0) {
+        // first half: hand the raw accumulator to the second half
+#pragma unroll 1
+        for (int c = 0; c < BN_MMA / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tb + c * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) part[(c * 32 + j) * 128 + prow] = __uint_as_float(v[j]);
+        }
+        __threadfence();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          flag_release(flag);
+          mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+        }
+        continue;
+      }
+      if (it.half == 1) {
+        // second half: wait (bounded) for the first half's partial
+        int ready = 1;
+        if (lane == 0) {
+          const unsigned long long t0 = globaltimer();
+          while (flag_acquire(flag) == 0) {
+            if (*abort || globaltimer() - t0 > kWaitTimeoutNs) {
+              if (!*abort) atomicOr(p.err, DEVERR_TIMEOUT | SITE_PAIR_EPILOGUE);
+              *abort = 1;
+              ready = 0;
+              break;
+            }
+            __nanosleep(256);
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ready, 0)) break;
+        __threadfence();
+      }
+      // adds the first half's partial to columns [c0, c0 + 32) of this row
+      auto add_partial = [&](uint32_t (&v)[32], int c0) {
+        if (it.half == 1) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            v[j] = __float_as_uint(__uint_as_float(v[j]) + __ldcg(part + (c0 + j) * 128 + prow));
+        }
+      };
       const int sw = GATHER ? 0 : swap_rows(st, p.swap_max, e, m_blk);
       if (sw) {
         // swapped tail: this thread's TMEM lane is one weight row (an output
@@ -536,6 +649,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t v[32];
             tmem_ld32(tb + c * 32, v);
             tmem_ld_wait();
+            add_partial(v, c * 32);
             // the low lane finishes tokens 32c..32c+15, the high lane 32c+16..32c+31
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -546,7 +660,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               const int tok = c * 32 + (hi ? 16 : 0) + j;
               if (fvalid && tok < sw)
                 p.out[static_cast<size_t>(row0 + tok) * p.n_out + f] =
-                    __float2bfloat16_rn(g / (1.f + __expf(-g)) * u);
+                    __float2bfloat16_rn(silu_bf16_epilogue(g) * u);
             }
           }
         } else {
@@ -559,6 +673,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t v[32];
             tmem_ld32(tb + c * 32, v);
             tmem_ld_wait();
+            add_partial(v, c * 32);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int tok = c * 32 + j;
@@ -585,6 +700,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld32(tb + c * 32, g);
           tmem_ld32(tb + 128 + c * 32, u);
           tmem_ld_wait();
+          add_partial(g, c * 32);
+          add_partial(u, 128 + c * 32);
           const int col0 = n_blk * 128 + c * 32;
           if (rvalid && col0 < p.n_out) {
             uint32_t w[16];
@@ -592,8 +709,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int j = 0; j < 16; ++j) {
               const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
               const float u0 = __uint_as_float(u[2 * j]), u1 = __uint_as_float(u[2 * j + 1]);
-              const float h0 = g0 / (1.f + __expf(-g0)) * u0;
-              const float h1 = g1 / (1.f + __expf(-g1)) * u1;
+              const float h0 = silu_bf16_epilogue(g0) * u0;
+              const float h1 = silu_bf16_epilogue(g1) * u1;
               w[j] = pack_bf16x2(h0, h1);
             }
             store_row32(rowp, col0, p.n_out, w);
@@ -605,6 +722,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint32_t v[32];
           tmem_ld32(tb + c * 32, v);
           tmem_ld_wait();
+          add_partial(v, c * 32);
           const int col0 = n_blk * 256 + c * 32;
           if (rvalid && col0 < p.n_out) {
             const float* bias = p.bias ? p.bias + static_cast<size_t>(e) * p.n_out + col0 : nullptr;
@@ -744,7 +862,8 @@ cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* 
                                 const int* offsets, int E, int Kdim, int N, int w_rows_per_expert,
                                 const float* bias, void* C, unsigned int* err, int* tile_counter,
                                 cudaStream_t s, const int* gather_perm, int gather_K,
-                                int gather_rows, int swap_max) {
+                                int gather_rows, int swap_max, float* split_partial,
+                                int* split_flags) {
   CUtensorMap ma, mb, mgu;
   TokMaps tok;
   const bool gather = gather_perm != nullptr;
@@ -778,6 +897,9 @@ cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* 
   p.err = err;
   p.swap_max = swap_max;
   p.tile_counter = tile_counter;
+  p.split_partial = split_flags ? split_partial : nullptr;
+  p.split_flags = split_flags;
+  p.split_cap = kSplitMaxCtas / 2;
   const int bn_out = (act == kSiluGated) ? 128 : 256;
   const long long tiles_bound =
       (static_cast<long long>(a_rows) / BMP + E) * ((N + bn_out - 1) / bn_out);

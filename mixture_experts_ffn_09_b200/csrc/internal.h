@@ -13,11 +13,20 @@ constexpr int kMaxExperts = 256;
 constexpr int kRouterTokensPerCta = 32;   // tokens per router CTA = per permute block
 constexpr int kTileM = 128;               // rows of one grouped-GEMM tile
 // Tile counters of the grouped GEMMs' dynamic schedulers, one per GEMM of a
-// forward, each on its own 128-byte line: kSchedInts ints in the workspace,
-// zeroed by the scatter kernel of the same forward.
-constexpr int kSchedInts = 64;
+// forward, each on its own 128-byte line, then each GEMM's flags of the
+// split last wave (one per split unit, CTA and epilogue warp): kSchedInts
+// ints in the workspace, zeroed by the scatter kernel of the same forward.
+constexpr int kSplitMaxCtas = 148;           // CTAs whose partial tiles the scratch holds
+constexpr int kSplitFlags = kSplitMaxCtas * 4;
 constexpr int kSchedGateUp = 0;
 constexpr int kSchedDown = 32;
+constexpr int kSchedFlagsGateUp = 64;
+constexpr int kSchedFlagsDown = kSchedFlagsGateUp + kSplitFlags;
+constexpr int kSchedInts = kSchedFlagsDown + kSplitFlags;
+// fp32 partial accumulators of the split last wave: 128 rows x 256 columns
+// per CTA of a split unit
+constexpr size_t kSplitCtaBytes = 128u * 256u * 4u;
+constexpr size_t kSplitBytes = kSplitMaxCtas * kSplitCtaBytes;
 
 enum DType : int { kF32 = 0, kBF16 = 1 };
 
@@ -114,11 +123,15 @@ cudaError_t launch_gemm_tc(int act, const void* A, int a_rows, const void* W, co
 // swapped-operand tile whose N is the block's rows rounded up to 16.  The
 // persistent pairs take tiles in order from *tile_counter, which must be
 // zero when the kernel starts (the scatter kernel zeroes it each forward).
+// split_partial (kSplitBytes) / split_flags (kSplitFlags, zero at start):
+// the last wave's units run as two halves of the k-blocks, the first
+// handing its fp32 accumulator to the second; null: no split.
 cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* W,
                                 const int* offsets, int E, int Kdim, int N, int w_rows_per_expert,
                                 const float* bias, void* C, unsigned int* err, int* tile_counter,
                                 cudaStream_t s, const int* gather_perm = nullptr,
-                                int gather_K = 0, int gather_rows = 0, int swap_max = 0);
+                                int gather_K = 0, int gather_rows = 0, int swap_max = 0,
+                                float* split_partial = nullptr, int* split_flags = nullptr);
 
 // The whole float32 forward of a small layer in one launch: a cluster with
 // one CTA per expert (router in every CTA, the expert's rows in its CTA,

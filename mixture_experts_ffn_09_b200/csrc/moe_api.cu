@@ -41,13 +41,15 @@ constexpr long long kScatterScansItself = 4096;
 cudaError_t launch_gemm_bf16(int act, const void* A, int a_rows, const void* W,
                              const int* offsets, int E, int T, int K, int Kdim, int N,
                              int w_rows, const float* bias, void* C, unsigned int* err,
-                             int* tile_counter, cudaStream_t s, const int* gather_perm = nullptr) {
+                             int* tile_counter, float* split_partial, int* split_flags,
+                             cudaStream_t s, const int* gather_perm = nullptr) {
   const int mode = g_gemm_mode.load();
   const bool pair = mode == MOE_GEMM_2SM ||
                     (mode == MOE_GEMM_AUTO && static_cast<long long>(T) * K >= 512LL * E);
   if (pair)
     return moe::launch_gemm_tc_pair(act, A, a_rows, W, offsets, E, Kdim, N, w_rows, bias, C, err,
-                                    tile_counter, s, gather_perm, K, T, g_tail_swap.load());
+                                    tile_counter, s, gather_perm, K, T, g_tail_swap.load(),
+                                    split_partial, split_flags);
   return moe::launch_gemm_tc(act, A, a_rows, W, offsets, E, static_cast<long long>(T) * K, Kdim, N,
                              w_rows, bias, C, err, s, gather_perm, K, T);
 }
@@ -236,7 +238,9 @@ struct StageTimer {
 
 // ------------------------------------------------------ workspace layout
 struct Layout {
-  size_t idx32, w32, bcount, bbase, totals, offsets, sched, perm, pos, bal, xperm, h, y, total;
+  size_t idx32, w32, bcount, bbase, totals, offsets, sched, perm, pos, bal, part, xperm, h, y,
+      total;
+  bool split;     // the CTA-pair GEMMs may split their last wave (scratch reserved)
   int B, Rpad;
 };
 
@@ -266,6 +270,10 @@ Layout layout(int64_t T, int64_t D, int64_t F, int E, int K, int elem) {
                           : moe::router_tc_parts(static_cast<int>(T));
     L.bal = take(sizeof(float) * 3 * static_cast<size_t>(parts) * E);
   }
+  // the split last wave's partial tiles, for layers whose automatic choice
+  // is the CTA-pair GEMM (bf16, at least 512 routed rows per expert)
+  L.split = elem == 2 && R >= 512LL * E;
+  L.part = take(L.split ? moe::kSplitBytes : 0);
   L.xperm = take(static_cast<size_t>(elem) * L.Rpad * D);
   L.h = take(static_cast<size_t>(elem) * L.Rpad * F);
   L.y = take(static_cast<size_t>(elem) * L.Rpad * D);
@@ -506,6 +514,7 @@ moe_status_t ffn_forward_impl(const void* x, const void* router, const void* gat
   void* H = ws + L.h;
   void* Y = ws + L.y;
   float* bal = reinterpret_cast<float*>(ws + L.bal);
+  float* part = L.split ? reinterpret_cast<float*>(ws + L.part) : nullptr;
   const float cap = opts ? opts->capacity_factor : 0.f;
   const int seq_len = opts ? static_cast<int>(opts->seq_len) : 0;
   float* balance_out = opts ? opts->balance : nullptr;
@@ -587,14 +596,16 @@ moe_status_t ffn_forward_impl(const void* x, const void* router, const void* gat
   if (dt == MOE_BF16) {
     e = timer.run(2, [&] {
       return launch_gemm_bf16(gu_act, fused_gather ? x : xperm, L.Rpad, gate_up_proj, offsets, E,
-                              Ti, K, Di, Fi, gu_rows, b1, H, dev->err, sched + moe::kSchedGateUp, s,
+                              Ti, K, Di, Fi, gu_rows, b1, H, dev->err, sched + moe::kSchedGateUp,
+                              part, part ? sched + moe::kSchedFlagsGateUp : nullptr, s,
                               fused_gather ? perm : nullptr);
     });
     if (e != cudaSuccess) return cuda_fail(e, "gate_up launch");
     if (!debug_wait(dev, s, "gate_up GEMM")) return MOE_ERR_TIMEOUT;
     e = timer.run(3, [&] {
       return launch_gemm_bf16(2, H, L.Rpad, down_proj, offsets, E, Ti, K, Fi, Di, Di, b2, Y,
-                              dev->err, sched + moe::kSchedDown, s);
+                              dev->err, sched + moe::kSchedDown, part,
+                              part ? sched + moe::kSchedFlagsDown : nullptr, s);
     });
     if (e != cudaSuccess) return cuda_fail(e, "down launch");
     if (!debug_wait(dev, s, "down GEMM")) return MOE_ERR_TIMEOUT;

@@ -176,9 +176,15 @@ def test_workspace_size(L):
     assert ws < 128 * (64 + 128 + 64) * 4 + 64 * 1024
     assert moe.workspace_size(64, 64, 128, 8, 9, moe.F32) == 0
     assert moe.workspace_size(64, 64, 128, 8, 2, moe.F64) == 0
+    # a layer in the CTA-pair regime (>= 512 routed rows per expert) also
+    # holds the split last wave's fp32 partial tiles: 148 CTAs x 128 x 256
+    split = 148 * 128 * 256 * 4
     big = moe.workspace_size(4096, 4096, 14336, 8, 2, moe.BF16)
-    assert big >= 8192 * (4096 + 14336 + 4096) * 2
-    assert big < 8192 * (4096 + 14336 + 4096) * 2 + 8 * 1024 * 1024
+    assert big >= 8192 * (4096 + 14336 + 4096) * 2 + split
+    assert big < 8192 * (4096 + 14336 + 4096) * 2 + split + 8 * 1024 * 1024
+    # decode-sized layers take no partial tiles
+    dec = moe.workspace_size(32, 4096, 14336, 8, 8, moe.BF16)
+    assert dec < 256 * (4096 + 14336 + 4096) * 2 + 1024 * 1024
 
 
 def test_route_opts_layout_matches_the_header(tmp_path):

@@ -530,6 +530,33 @@ def test_small_float32_layer_runs_as_one_kernel(name):
     PL.check_out(res[0]["out"][same], res[1]["out"][same], "f32", "one kernel vs six")
 
 
+@pytest.mark.parametrize("act", ["silu_gated", "relu"])
+def test_split_last_wave(act):
+    """Layers in the CTA-pair regime run their last wave as k-halves: the
+    first half of a tile hands its fp32 accumulator to the second.  Here every
+    tile is split (18 tiles, fewer than the pairs), the experts end in swapped
+    tails, and every token is compared with the oracle; the result repeats
+    bit for bit and equals the fused-gather variant's."""
+    from mixture_experts_ffn_09_b200 import moe
+    T, D, F, E, K = 1200, 256, 384, 2, 1       # 1200 routed rows >= 512 per expert
+    d = synth.random_case(501, T, D, F, E, act=act, dtype="bf16", weight_std=0.05)
+    g, _ = _full_check(d, E, K, True, act, "bf16")
+    load = np.bincount(g["sel"].ravel(), minlength=E)
+    assert (load % 256 > 0).all() and (load % 256 <= 128).any()   # a swapped tail
+    dev = PL.to_device(d)
+    a = PL.run_gpu(dev, E, K, True, act)
+    b = PL.run_gpu(dev, E, K, True, act)
+    prev = moe.set_fused_gather(True)
+    try:
+        c = PL.run_gpu(dev, E, K, True, act)
+    finally:
+        moe.set_fused_gather(prev)
+    for k in ("out", "sel", "w"):
+        np.testing.assert_array_equal(a[k], b[k])
+        np.testing.assert_array_equal(a[k], c[k])
+        np.testing.assert_array_equal(a[k], g[k])
+
+
 def _random_shapes(n, seed):
     """Seeded layer shapes across the supported ranges: bf16 needs D and F
     multiples of 8, any sizes on float32."""
