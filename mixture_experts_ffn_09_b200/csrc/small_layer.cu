@@ -35,8 +35,8 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kRowGroup = 8;      // rows of one expert computed together by a thread
+constexpr int kThreads = 512;
+constexpr int kRowGroup = 4;      // rows of one expert computed together by a thread
 
 struct SmallParams {
   const float* x;
@@ -57,28 +57,37 @@ struct SmallParams {
 // cluster so that a remote Y row is at the same offset as a local one.
 struct SmallLayout {
   int xs, wr, lg, sel, w, rank, tok, wcnt, w1, w2, h, y, total;   // offsets in 4-byte words
-  int ldx, ldw1, ldw2;                                            // padded row lengths
+  int ldx, ldw1, ldw2, ldh;                                       // padded row lengths
 };
 
+__host__ __device__ constexpr int round4(int v) { return (v + 3) & ~3; }
+
+// Rows read whole by every lane at once (x, the router, H) are padded to a
+// multiple of 4 floats, so they are read 16 bytes at a time (one wavefront
+// serves all lanes); x and router rows get 4 more so that a warp reading 4
+// different rows at once hits different banks.  Weight rows, read one
+// element per lane along a column, keep an odd length: conflict-free.
+// Every region starts on a 16-byte boundary.
 __host__ __device__ inline SmallLayout small_layout(int T, int D, int F, int E, int K, int gated) {
   SmallLayout L;
   const int gu_rows = gated ? 2 * F : F;
-  L.ldx = D + 1;          // odd row lengths keep column walks free of bank conflicts
+  L.ldx = round4(D) + 4;
   L.ldw1 = D + 1;
   L.ldw2 = F + 1;
+  L.ldh = round4(F);
   int o = 0;
-  L.xs = o;   o += T * L.ldx;
-  L.wr = o;   o += E * L.ldx;
-  L.lg = o;   o += T * E;
-  L.sel = o;  o += T * K;
-  L.w = o;    o += T * K;
-  L.rank = o; o += T * K;
-  L.tok = o;  o += T;
-  L.wcnt = o; o += (kThreads / 32) * kSmallMaxExperts;
-  L.w1 = o;   o += gu_rows * L.ldw1;
-  L.w2 = o;   o += D * L.ldw2;
-  L.h = o;    o += T * F;
-  L.y = o;    o += T * D;
+  L.xs = o;   o += round4(T * L.ldx);
+  L.wr = o;   o += round4(E * L.ldx);
+  L.lg = o;   o += round4(T * E);
+  L.sel = o;  o += round4(T * K);
+  L.w = o;    o += round4(T * K);
+  L.rank = o; o += round4(T * K);
+  L.tok = o;  o += round4(T);
+  L.wcnt = o; o += round4((kThreads / 32) * kSmallMaxExperts);
+  L.w1 = o;   o += round4(gu_rows * L.ldw1);
+  L.w2 = o;   o += round4(D * L.ldw2);
+  L.h = o;    o += round4(T * L.ldh);
+  L.y = o;    o += round4(T * D);
   L.total = o;
   return L;
 }
@@ -131,7 +140,7 @@ __device__ __forceinline__ bool ranks_before(float v, int e, float bv, int be) {
 
 template <bool kGated>
 __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const SmallParams p) {
-  extern __shared__ float sm[];
+  extern __shared__ __align__(16) float sm[];
   const int T = p.T, D = p.D, F = p.F, E = p.E, K = p.K;
   const SmallLayout L = small_layout(T, D, F, E, K, kGated);
   float* xs = sm + L.xs;
@@ -171,10 +180,12 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     int d = 0;
     for (; d + 4 <= D; d += 4) {
-      a0 = fmaf(xr[d], rr[d], a0);
-      a1 = fmaf(xr[d + 1], rr[d + 1], a1);
-      a2 = fmaf(xr[d + 2], rr[d + 2], a2);
-      a3 = fmaf(xr[d + 3], rr[d + 3], a3);
+      const float4 xv = *reinterpret_cast<const float4*>(xr + d);
+      const float4 rv = *reinterpret_cast<const float4*>(rr + d);
+      a0 = fmaf(xv.x, rv.x, a0);
+      a1 = fmaf(xv.y, rv.y, a1);
+      a2 = fmaf(xv.z, rv.z, a2);
+      a3 = fmaf(xv.w, rv.w, a3);
     }
     for (; d < D; ++d) a0 = fmaf(xr[d], rr[d], a0);
     float acc = (a0 + a1) + (a2 + a3);
@@ -263,8 +274,36 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
       const int r = g * kRowGroup + j;
       xr[j] = xs + (r < rows ? tok[r] : 0) * L.ldx;
     }
-#pragma unroll 4
-    for (int d = 0; d < D; ++d) {
+    // x rows four columns at a time (16-byte reads every lane shares)
+    int d = 0;
+#pragma unroll 2
+    for (; d + 4 <= D; d += 4) {
+      float4 xv[kRowGroup];
+#pragma unroll
+      for (int j = 0; j < kRowGroup; ++j) xv[j] = *reinterpret_cast<const float4*>(xr[j] + d);
+      const float va[4] = {wa[d], wa[d + 1], wa[d + 2], wa[d + 3]};
+      float vb[4] = {0.f, 0.f, 0.f, 0.f};
+      if (kGated) {
+        vb[0] = wb[d];
+        vb[1] = wb[d + 1];
+        vb[2] = wb[d + 2];
+        vb[3] = wb[d + 3];
+      }
+#pragma unroll
+      for (int j = 0; j < kRowGroup; ++j) {
+        a[j] = fmaf(xv[j].x, va[0], a[j]);
+        a[j] = fmaf(xv[j].y, va[1], a[j]);
+        a[j] = fmaf(xv[j].z, va[2], a[j]);
+        a[j] = fmaf(xv[j].w, va[3], a[j]);
+        if (kGated) {
+          b[j] = fmaf(xv[j].x, vb[0], b[j]);
+          b[j] = fmaf(xv[j].y, vb[1], b[j]);
+          b[j] = fmaf(xv[j].z, vb[2], b[j]);
+          b[j] = fmaf(xv[j].w, vb[3], b[j]);
+        }
+      }
+    }
+    for (; d < D; ++d) {
       const float va = wa[d];
       const float vb = kGated ? wb[d] : 0.f;
 #pragma unroll
@@ -279,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
     for (int j = 0; j < kRowGroup; ++j) {
       const int r = g * kRowGroup + j;
       if (r < rows)
-        hs[r * F + f] = kGated ? a[j] / (1.f + expf(-a[j])) * b[j] : fmaxf(a[j] + bias, 0.f);
+        hs[r * L.ldh + f] = kGated ? a[j] / (1.f + expf(-a[j])) * b[j] : fmaxf(a[j] + bias, 0.f);
     }
   }
   __syncthreads();
@@ -291,9 +330,21 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
     const float* wd = w2 + d * L.ldw2;
     const float* hr[kRowGroup];
 #pragma unroll
-    for (int j = 0; j < kRowGroup; ++j) hr[j] = hs + min(g * kRowGroup + j, rows - 1) * F;
-#pragma unroll 4
-    for (int f = 0; f < F; ++f) {
+    for (int j = 0; j < kRowGroup; ++j) hr[j] = hs + min(g * kRowGroup + j, rows - 1) * L.ldh;
+    int f = 0;
+#pragma unroll 2
+    for (; f + 4 <= F; f += 4) {
+      const float v[4] = {wd[f], wd[f + 1], wd[f + 2], wd[f + 3]};
+#pragma unroll
+      for (int j = 0; j < kRowGroup; ++j) {
+        const float4 h4 = *reinterpret_cast<const float4*>(hr[j] + f);
+        a[j] = fmaf(h4.x, v[0], a[j]);
+        a[j] = fmaf(h4.y, v[1], a[j]);
+        a[j] = fmaf(h4.z, v[2], a[j]);
+        a[j] = fmaf(h4.w, v[3], a[j]);
+      }
+    }
+    for (; f < F; ++f) {
       const float v = wd[f];
 #pragma unroll
       for (int j = 0; j < kRowGroup; ++j) a[j] = fmaf(hr[j][f], v, a[j]);
