@@ -165,6 +165,7 @@ struct Tail {
   int total_tiles;
   int tile_start[kMaxExperts + 1];
   int off[kMaxExperts + 1];
+  uint32_t wfast[(kMaxExperts + 31) / 32];   // bit e: expert e's tiles go weight block fastest
 };
 
 constexpr size_t kSmemBytes = STAGES * STAGE_BYTES + sizeof(Tail);
@@ -262,6 +263,13 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
       : "memory");
 }
 
+// Expert, row block and weight block of tile t.  An expert's tiles are
+// ordered with the row block fastest (consecutive tiles share a weight
+// block, and the expert's token rows are re-read for every weight block),
+// or, for an expert with more token rows than weight rows, with the weight
+// block fastest (consecutive tiles share the token rows, and the smaller
+// weights are the operand re-read).  Either way the operand that must stay
+// in L2 between its uses is the smaller one.
 __device__ __forceinline__ void decode_tile(const Tail* st, int E, int n_tiles, int t, int& e,
                                             int& m_blk, int& n_blk) {
   int lo = 0, hi = E - 1;
@@ -271,9 +279,14 @@ __device__ __forceinline__ void decode_tile(const Tail* st, int E, int n_tiles, 
   }
   e = lo;
   const int local = t - st->tile_start[e];
-  const int mt = (st->tile_start[e + 1] - st->tile_start[e]) / n_tiles;
-  n_blk = local / mt;
-  m_blk = local - n_blk * mt;
+  if ((st->wfast[e >> 5] >> (e & 31)) & 1u) {
+    m_blk = local / n_tiles;
+    n_blk = local - m_blk * n_tiles;
+  } else {
+    const int mt = (st->tile_start[e + 1] - st->tile_start[e]) / n_tiles;
+    n_blk = local / mt;
+    m_blk = local - n_blk * mt;
+  }
 }
 
 // Rows of a swapped tail tile (1..255), or 0 for a regular tile.  Every row
@@ -363,12 +376,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   pdl_wait();
   if (threadIdx.x == 0) {
     int acc = 0;
+    for (int j = 0; j < (kMaxExperts + 31) / 32; ++j) st->wfast[j] = 0u;
     for (int e = 0; e < E; ++e) {
       const int o0 = p.offsets[e], o1 = p.offsets[e + 1];
       const int mt = (o1 - o0 + BMP - 1) / BMP;
       st->off[e] = o0;
       st->tile_start[e] = acc;
       acc += mt * n_tiles;
+      if (o1 - o0 > p.b_rows) st->wfast[e >> 5] |= 1u << (e & 31);
     }
     st->off[E] = p.offsets[E];
     st->tile_start[E] = acc;
