@@ -9,9 +9,10 @@
 // pair stages its own 128 rows of A and HALF of the 256 B rows, and the pair's
 // MMA reads both CTAs' shared memory, so a CTA moves 32 KB per k-block for
 // the same 128 x 256 x 64 product that costs 48 KB on one CTA.  The saved
-// shared memory buys a 7-stage ring (224 KB: the ring starts at the
+// shared memory buys a 6-stage ring (192 KB: the ring starts at the
 // 1024-byte-aligned base of dynamic shared memory, and the tile table keeps
-// only the per-expert tile starts and row offsets).
+// only the per-expert tile starts and row offsets) and 8 KB of output
+// staging per epilogue warp.
 //
 // Cluster of 2 CTAs (rank 0 = leader), 192 threads each:
 //   warp 0 (both)   TMA producer for this CTA's A rows and B half; the loads
@@ -21,9 +22,13 @@
 //                   (tcgen05.alloc.cta_group::2); in the leader one lane
 //                   issues the pair's MMAs and commits, multicast to both
 //                   CTAs, the stage releases and accumulator completions;
-//   warps 2..5      epilogue of this CTA's 128 rows, as in gemm_tc.cu; each
-//                   warp's release of an accumulator arrives on the
-//                   leader's barrier (8 arrivals per tile).
+//   warps 2..5      epilogue of this CTA's 128 rows; each warp's release of
+//                   an accumulator arrives on the leader's barrier (8
+//                   arrivals per tile).  A warp converts 128 columns of its
+//                   32 rows (a row per lane, as TMEM hands them out) into
+//                   its staging area, then stores them as whole 256-byte
+//                   row runs, two rows per instruction: 4 full lines per
+//                   store instead of 32 scattered 16-byte pieces.
 // For the gated expert the leader stages the 128 gate rows and the peer the
 // matching 128 up rows, so accumulator columns [0,128) are gate and
 // [128,256) up in both CTAs, exactly as in the one-CTA kernel.
@@ -74,7 +79,7 @@ constexpr int BMC = 128;                      // rows per CTA
 constexpr int BMP = 256;                      // rows per pair
 constexpr int BK = 64;
 constexpr int BN_MMA = 256;
-constexpr int STAGES = 7;
+constexpr int STAGES = 6;
 constexpr int A_BYTES = BMC * BK * 2;         // 16 KB
 constexpr int B_BYTES = (BN_MMA / 2) * BK * 2;  // 16 KB (this CTA's half)
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -168,7 +173,33 @@ struct Tail {
   uint32_t wfast[(kMaxExperts + 31) / 32];   // bit e: expert e's tiles go weight block fastest
 };
 
-constexpr size_t kSmemBytes = STAGES * STAGE_BYTES + sizeof(Tail);
+constexpr size_t kTailBytes = (sizeof(Tail) + 127) & ~size_t(127);
+constexpr int kEpiStageBytes = 32 * 256;      // per epilogue warp: 32 rows x 256 B
+constexpr size_t kSmemBytes = STAGES * STAGE_BYTES + kTailBytes + 4 * kEpiStageBytes;
+
+// Rows of 256 B staged by the epilogue warp, 16-byte unit u of row r at
+// unit u ^ (r & 7): the row-per-lane writes and the run-per-half-warp reads
+// are both free of bank conflicts.
+__device__ __forceinline__ void epi_put(uint8_t* stg, int r, int u, const uint32_t* w) {
+  *reinterpret_cast<uint4*>(stg + r * 256 + ((u ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+// Stores the staged 32 x 128 block: each instruction writes two 256-byte row
+// runs.  Rows at or beyond row_end and columns at or beyond n_out are skipped.
+__device__ __forceinline__ void epi_flush(const uint8_t* stg, int lane, __nv_bfloat16* out, int grow0,
+                                          int row_end, int col_base, int n_out) {
+  __syncwarp();
+  const int u = lane & 15;
+  const int col = col_base + u * 8;
+#pragma unroll 4
+  for (int i = 0; i < 16; ++i) {
+    const int r = 2 * i + (lane >> 4);
+    const uint4 v = *reinterpret_cast<const uint4*>(stg + r * 256 + ((u ^ (r & 7)) << 4));
+    const int grow = grow0 + r;
+    if (grow < row_end && col < n_out)
+      *reinterpret_cast<uint4*>(out + static_cast<size_t>(grow) * n_out + col) = v;
+  }
+  __syncwarp();
+}
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -334,6 +365,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
   Tail* st = reinterpret_cast<Tail*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* epi_stage = smem + STAGES * STAGE_BYTES + kTailBytes;
 
   constexpr int BN_OUT = (EPI == kSiluGated) ? 128 : 256;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -705,9 +737,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
         continue;
       }
-      const int grow = st->off[e] + m_blk * BMP + static_cast<int>(rank) * BMC + lane_base + lane;
-      const bool rvalid = grow < st->off[e + 1];
-      __nv_bfloat16* rowp = p.out + static_cast<size_t>(rvalid ? grow : 0) * p.n_out;
+      const int grow0 = st->off[e] + m_blk * BMP + static_cast<int>(rank) * BMC + lane_base;
+      const int row_end = st->off[e + 1];
+      uint8_t* stg = epi_stage + (warp - 2) * kEpiStageBytes;
       if (EPI == kSiluGated) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -717,29 +749,28 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld_wait();
           add_partial(g, c * 32);
           add_partial(u, 128 + c * 32);
-          const int col0 = n_blk * 128 + c * 32;
-          if (rvalid && col0 < p.n_out) {
-            uint32_t w[16];
+          uint32_t w[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
-              const float u0 = __uint_as_float(u[2 * j]), u1 = __uint_as_float(u[2 * j + 1]);
-              const float h0 = silu_bf16_epilogue(g0) * u0;
-              const float h1 = silu_bf16_epilogue(g1) * u1;
-              w[j] = pack_bf16x2(h0, h1);
-            }
-            store_row32(rowp, col0, p.n_out, w);
+          for (int j = 0; j < 16; ++j) {
+            const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
+            const float u0 = __uint_as_float(u[2 * j]), u1 = __uint_as_float(u[2 * j + 1]);
+            w[j] = pack_bf16x2(silu_bf16_epilogue(g0) * u0, silu_bf16_epilogue(g1) * u1);
           }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) epi_put(stg, lane, c * 4 + q, w + 4 * q);
         }
+        epi_flush(stg, lane, p.out, grow0, row_end, n_blk * 128, p.n_out);
       } else {
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tb + c * 32, v);
-          tmem_ld_wait();
-          add_partial(v, c * 32);
-          const int col0 = n_blk * 256 + c * 32;
-          if (rvalid && col0 < p.n_out) {
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            const int c = h * 4 + cc;
+            uint32_t v[32];
+            tmem_ld32(tb + c * 32, v);
+            tmem_ld_wait();
+            add_partial(v, c * 32);
+            const int col0 = n_blk * 256 + c * 32;
             const float* bias = p.bias ? p.bias + static_cast<size_t>(e) * p.n_out + col0 : nullptr;
             uint32_t w[16];
 #pragma unroll
@@ -755,8 +786,10 @@ __global__ void __launch_bounds__(THREADS, 1)
               }
               w[j] = pack_bf16x2(a0, a1);
             }
-            store_row32(rowp, col0, p.n_out, w);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) epi_put(stg, lane, cc * 4 + q, w + 4 * q);
           }
+          epi_flush(stg, lane, p.out, grow0, row_end, n_blk * 256 + h * 128, p.n_out);
         }
       }
       tc_fence_before();
