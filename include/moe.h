@@ -289,6 +289,21 @@ MOE_API int moe_set_gemm_mode(int mode);
 MOE_API int moe_set_tail_swap(int max_rows);
 
 /*
+ * Cluster size of the one-kernel float32 small layer (process-wide
+ * setting).  A small float32 layer (E <= 8, T*K <= 256, no routing
+ * options, the kernel's shared memory within 200 KB) runs as one cluster
+ * of CTAs; each expert's hidden columns are split over CTAs in proportion
+ * to the rows it received.  ctas: MOE_SMALL_CLUSTER_AUTO (16 where the GPU
+ * can co-schedule a cluster of 16 such CTAs, else 8), 8 or 16.  A forced
+ * 16 on a GPU that cannot co-schedule it makes the forward fail with
+ * MOE_ERR_CUDA.  Results agree across sizes up to fp32 summation order.
+ * Returns the previous setting, or -1 for any other value (nothing
+ * changes).
+ */
+#define MOE_SMALL_CLUSTER_AUTO 0
+MOE_API int moe_set_small_cluster(int ctas);
+
+/*
  * Whether the bf16 gate_up GEMM fetches its token rows from x by index
  * (TMA tile::gather4, four rows per copy) instead of from an expert-sorted
  * copy written by a separate gather kernel.  Results are bit-identical.

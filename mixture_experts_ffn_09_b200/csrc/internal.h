@@ -133,19 +133,22 @@ cudaError_t launch_gemm_tc_pair(int act, const void* A, int a_rows, const void* 
                                 int gather_K = 0, int gather_rows = 0, int swap_max = 0,
                                 float* split_partial = nullptr, int* split_flags = nullptr);
 
-// The whole float32 forward of a small layer in one launch: a cluster with
-// one CTA per expert (router in every CTA, the expert's rows in its CTA,
-// the combine over distributed shared memory).  For layers within these
-// limits and no routing options.
-constexpr int kSmallMaxExperts = 8;             // one portable cluster
+// The whole float32 forward of a small layer in one launch: a cluster of
+// 8 or 16 CTAs (router in every CTA; each expert's hidden columns split
+// over CTAs in proportion to its rows; the combine over distributed shared
+// memory).  For layers within these limits and no routing options.
+constexpr int kSmallMaxExperts = 8;
+constexpr int kSmallMinCluster = 8;             // the portable cluster size
+constexpr int kSmallMaxCluster = 16;            // where the GPU co-schedules 16 CTAs
 constexpr int kSmallMaxRows = 256;              // routed rows T*K
 constexpr size_t kSmallMaxSmem = 200u << 10;    // x, router, one expert's weights, H, Y
 bool small_layer_fits(int T, int D, int F, int E, int K, int gated);
+// cluster: 0 = automatic (16 where possible, else 8), or 8 / 16.
 cudaError_t launch_small_layer_f32(const float* x, const float* router, const float* rb,
                                    const float* gu, const float* dn, const float* b1,
                                    const float* b2, int T, int D, int F, int E, int K, int norm,
                                    int gated, float* out, int64_t* sel64, float* wout,
-                                   float* logits, cudaStream_t s);
+                                   float* logits, int cluster, cudaStream_t s);
 
 int num_sms();
 unsigned long long kernel_launches();   // accepted launches so far (note_launch)

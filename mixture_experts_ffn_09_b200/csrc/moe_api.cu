@@ -28,6 +28,7 @@ thread_local std::string g_last_error;
 
 std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
 std::atomic<int> g_tail_swap{MOE_TAIL_SWAP_DEFAULT};
+std::atomic<int> g_small_cluster{MOE_SMALL_CLUSTER_AUTO};
 std::atomic<int> g_fused_gather{0};
 std::atomic<int> g_pdl{0};   // programmatic dependent launch: opt-in
 std::atomic<int> g_debug_sync_ms{0};   // > 0: bounded wait after every kernel of a forward
@@ -357,6 +358,11 @@ int moe_set_tail_swap(int max_rows) {
   return g_tail_swap.exchange(max_rows);
 }
 
+int moe_set_small_cluster(int ctas) {
+  if (ctas != MOE_SMALL_CLUSTER_AUTO && ctas != 8 && ctas != 16) return -1;
+  return g_small_cluster.exchange(ctas);
+}
+
 const char* moe_last_error(void) { return g_last_error.c_str(); }
 
 const char* moe_status_string(moe_status_t s) {
@@ -535,7 +541,7 @@ moe_status_t ffn_forward_impl(const void* x, const void* router, const void* gat
           static_cast<const float*>(x), static_cast<const float*>(router), router_bias,
           static_cast<const float*>(gate_up_proj), static_cast<const float*>(down_proj), b1, b2,
           Ti, Di, Fi, E, K, norm_topk_prob ? 1 : 0, gu_act == 0 ? 1 : 0, static_cast<float*>(out),
-          selected_experts, routing_weights, router_logits, s);
+          selected_experts, routing_weights, router_logits, g_small_cluster.load(), s);
     });
     if (e != cudaSuccess) return cuda_fail(e, "small-layer launch");
     if (!debug_wait(dev, s, "small layer")) return MOE_ERR_TIMEOUT;

@@ -4,8 +4,8 @@
 // "Problem": T=64 tokens, D=32, F=64, E=4 Dense/ReLU experts with biases) and
 // of mojolearn.MoEBlock's example (64 tokens, D=64, F=128, E=8, SiLU-gated)
 // are a few MFLOP: the six kernels of the general path cost far more in
-// launches than in work.  Here one thread-block cluster with one CTA per
-// expert does everything:
+// launches than in work.  Here one thread-block cluster of C CTAs (16 where
+// the GPU can co-schedule them, else 8) does everything:
 //
 //   1. every CTA computes the router for all tokens - logits (+ bias),
 //      softmax, top-k (descending, equal logits to the lower index, as the
@@ -13,17 +13,29 @@
 //      the weights of "Weight the selected outputs" - with the same code on
 //      the same data, so all CTAs agree on the selection bit for bit; CTA 0
 //      writes the routing outputs;
-//   2. CTA e lists the tokens that chose expert e in token order, stages
-//      that expert's weights in shared memory and computes its rows:
-//      H = silu(x Wg^T) * (x Wu^T), or relu(x W1^T + b1), then Y = H Wd^T
-//      (+ b2), in fp32 FMA;
-//   3. after a cluster barrier each CTA combines a slice of the tokens:
-//      out[t] = sum_k w[t, k] * Y_{e_k}[row of t in e_k], the k-th term read
-//      from expert e_k's CTA through distributed shared memory, summed in
-//      slot order and written once.
+//   2. from the rows each expert received, every CTA derives the same
+//      assignment of the C CTAs to experts: each expert with rows gets one
+//      CTA, and each further CTA goes to the expert with the most rows per
+//      CTA (lower index on ties).  An expert's s CTAs split its hidden
+//      columns F into s slices of whole 4-column groups, so the routing skew
+//      of a real batch (one expert can take almost half of all rows) is
+//      spread over several SMs instead of setting the time of the launch;
+//   3. the CTA holding slice [f0, f1) of expert e stages that slice of the
+//      weights (gate and up rows f0..f1-1 of gate_up_proj[e], columns
+//      f0..f1-1 of down_proj[e]), lists the tokens that chose e in token
+//      order, and computes H[:, f0:f1] = silu(x Wg^T) * (x Wu^T), or
+//      relu(x W1^T + b1), then the slice's share of Y = H Wd^T (+ b2 in the
+//      first slice), in fp32 FMA;
+//   4. after a cluster barrier each CTA combines a range of tokens:
+//      out[t] = sum_k w[t, k] * (sum over the slices of expert e_k of that
+//      slice's share of Y), each share read from its CTA through distributed
+//      shared memory, summed in slot order and slice order and written once.
 //
 // Same results as the general path up to fp32 summation order (the same
 // definitions, fp32 accumulation throughout); deterministic, no atomics.
+// At entry every CTA also asks L2 to prefetch its share of all experts'
+// weights, so that weights not yet in L2 come from DRAM while the router
+// runs.
 
 #include <math.h>
 
@@ -36,6 +48,7 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
 constexpr int kRowGroup = 4;      // rows of one expert computed together by a thread
 
 struct SmallParams {
@@ -50,44 +63,47 @@ struct SmallParams {
   int64_t* sel64;
   float* wout;
   float* logits;
-  int T, D, F, E, K, norm, gated;
-};
-
-// Shared-memory layout (floats / ints), the same in every CTA of the
-// cluster so that a remote Y row is at the same offset as a local one.
-struct SmallLayout {
-  int xs, wr, lg, sel, w, rank, tok, wcnt, w1, w2, h, y, total;   // offsets in 4-byte words
-  int ldx, ldw1, ldw2, ldh;                                       // padded row lengths
+  int T, D, F, E, K, norm;
+  int C;      // CTAs in the cluster
+  int vec;    // D and F multiples of 4: 16-byte copies
 };
 
 __host__ __device__ constexpr int round4(int v) { return (v + 3) & ~3; }
+// Length of rows that the lanes of a warp read 16 bytes at a time, each lane
+// from its own row: a multiple of 4 floats with an odd number of 16-byte
+// units, so the 8 lanes of a quarter warp fall in 8 different bank groups.
+__host__ __device__ constexpr int ld_odd4(int v) {
+  return ((round4(v) >> 2) & 1) ? round4(v) : round4(v) + 4;
+}
 
-// Rows read whole by every lane at once (x, the router, H) are padded to a
-// multiple of 4 floats, so they are read 16 bytes at a time (one wavefront
-// serves all lanes); x and router rows get 4 more so that a warp reading 4
-// different rows at once hits different banks.  Weight rows, read one
-// element per lane along a column, keep an odd length: conflict-free.
-// Every region starts on a 16-byte boundary.
+// Shared-memory layout (offsets in 4-byte words), the same in every CTA of
+// the cluster so that a remote Y row is at the same offset as a local one.
+// The weight, H and Y regions are sized for the largest case: one slice of
+// all F columns, an expert chosen by all T tokens.
+struct SmallLayout {
+  int xs, wr, lg, sel, w, rank, tok, wcnt, cfirst, scount, w1, w2, h, y, total;
+  int ldx;    // rows of x, of the router and of the staged gate/up weights
+};
+
 __host__ __device__ inline SmallLayout small_layout(int T, int D, int F, int E, int K, int gated) {
   SmallLayout L;
-  const int gu_rows = gated ? 2 * F : F;
-  L.ldx = round4(D) + 4;
-  L.ldw1 = D + 1;
-  L.ldw2 = F + 1;
-  L.ldh = round4(F);
+  L.ldx = ld_odd4(D);
+  const int fmax = round4(F);
   int o = 0;
-  L.xs = o;   o += round4(T * L.ldx);
-  L.wr = o;   o += round4(E * L.ldx);
-  L.lg = o;   o += round4(T * E);
-  L.sel = o;  o += round4(T * K);
-  L.w = o;    o += round4(T * K);
-  L.rank = o; o += round4(T * K);
-  L.tok = o;  o += round4(T);
-  L.wcnt = o; o += round4((kThreads / 32) * kSmallMaxExperts);
-  L.w1 = o;   o += round4(gu_rows * L.ldw1);
-  L.w2 = o;   o += round4(D * L.ldw2);
-  L.h = o;    o += round4(T * L.ldh);
-  L.y = o;    o += round4(T * D);
+  L.xs = o;     o += round4(T * L.ldx);
+  L.wr = o;     o += round4(E * L.ldx);
+  L.lg = o;     o += round4(T * E);
+  L.sel = o;    o += round4(T * K);
+  L.w = o;      o += round4(T * K);
+  L.rank = o;   o += round4(T * K);
+  L.tok = o;    o += round4(T);
+  L.wcnt = o;   o += kWarps * kSmallMaxExperts;
+  L.cfirst = o; o += kSmallMaxExperts;
+  L.scount = o; o += kSmallMaxExperts;
+  L.w1 = o;     o += (gated ? 2 : 1) * fmax * L.ldx;
+  L.w2 = o;     o += D * ld_odd4(F);
+  L.h = o;      o += T * fmax;
+  L.y = o;      o += round4(T * D);
   L.total = o;
   return L;
 }
@@ -113,24 +129,56 @@ __device__ __forceinline__ unsigned int lanemask_lt() {
   return m;
 }
 
-// Asynchronous 4-byte copies from global into shared memory: every copy of
-// a matrix is in flight at once and no registers hold the data.
+// Asynchronous copies from global into shared memory: every copy of a
+// matrix is in flight at once and no registers hold the data.
 __device__ __forceinline__ void cp_async4(float* dst, const float* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Starts copying a rows x cols block (source rows src_ld floats apart) into
+// shared rows of length ld.  vec: cols, src_ld, ld and both addresses are
+// multiples of 4 floats (16-byte copies); otherwise 4-byte copies.
+__device__ __forceinline__ void stage_async(float* dst, int ld, const float* __restrict__ src,
+                                            int src_ld, int rows, int cols, bool vec) {
+  if (vec) {
+    const int c4 = cols >> 2;
+    for (int i = threadIdx.x; i < rows * c4; i += kThreads) {
+      const int r = i / c4, c = (i - r * c4) << 2;
+      cp_async16(dst + r * ld + c, src + static_cast<size_t>(r) * src_ld + c);
+    }
+  } else {
+    for (int i = threadIdx.x; i < rows * cols; i += kThreads) {
+      const int r = i / cols, c = i - r * cols;
+      cp_async4(dst + r * ld + c, src + static_cast<size_t>(r) * src_ld + c);
+    }
+  }
 }
 
-// Starts copying a rows x cols row-major matrix into shared rows of length
-// ld: a warp per row, lanes along the row (coalesced).
-__device__ __forceinline__ void stage_async(float* dst, int ld, const float* __restrict__ src,
-                                            int rows, int cols) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int r = warp; r < rows; r += kThreads / 32)
-    for (int c = lane; c < cols; c += 32) cp_async4(dst + r * ld + c, src + static_cast<size_t>(r) * cols + c);
+// Asks L2 to fetch bytes [lo, hi) of the buffer at base (base, lo and hi
+// multiples of 16), in pieces of at most 16 KB spread over the warp's lanes.
+__device__ __forceinline__ void prefetch_l2(const void* base, size_t lo, size_t hi, int lane) {
+  constexpr size_t kPiece = 16384;
+  for (size_t off = lo + static_cast<size_t>(lane) * kPiece; off < hi; off += 32 * kPiece) {
+    const size_t n = hi - off < kPiece ? hi - off : kPiece;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(static_cast<const char*>(base) + off),
+                 "r"(static_cast<uint32_t>(n))
+                 : "memory");
+  }
+}
+
+// This CTA's share [lo, hi) of a buffer of `bytes` bytes (a multiple of
+// 16) split into C shares of whole 16-byte units; empty when lo >= hi.
+__device__ __forceinline__ void share_of(size_t bytes, int C, int me, size_t& lo, size_t& hi) {
+  const size_t units = bytes >> 4;
+  const size_t per = (units + C - 1) / C;
+  lo = per * me * 16;
+  hi = per * (me + 1) * 16;
+  if (hi > bytes) hi = bytes;
 }
 
 // True when (v, e) ranks before (bv, be): larger value, then lower index.
@@ -141,7 +189,8 @@ __device__ __forceinline__ bool ranks_before(float v, int e, float bv, int be) {
 template <bool kGated>
 __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const SmallParams p) {
   extern __shared__ __align__(16) float sm[];
-  const int T = p.T, D = p.D, F = p.F, E = p.E, K = p.K;
+  const int T = p.T, D = p.D, F = p.F, E = p.E, K = p.K, C = p.C;
+  const bool vec = p.vec != 0;
   const SmallLayout L = small_layout(T, D, F, E, K, kGated);
   float* xs = sm + L.xs;
   float* wr = sm + L.wr;
@@ -151,25 +200,31 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
   int* rank = reinterpret_cast<int*>(sm + L.rank);
   int* tok = reinterpret_cast<int*>(sm + L.tok);
   int* wcnt = reinterpret_cast<int*>(sm + L.wcnt);
+  int* cfirst = reinterpret_cast<int*>(sm + L.cfirst);
+  int* scount = reinterpret_cast<int*>(sm + L.scount);
   float* w1 = sm + L.w1;
   float* w2 = sm + L.w2;
   float* hs = sm + L.h;
   float* ys = sm + L.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int me = static_cast<int>(cta_rank());      // this CTA's expert
+  const int me = static_cast<int>(cta_rank());
   const int gu_rows = kGated ? 2 * F : F;
 
   pdl_trigger();
   pdl_wait();
-  // ---- stage x and the router (group 0), then this expert's weights
-  // (group 1), which land while the router runs
-  stage_async(xs, L.ldx, p.x, T, D);
-  stage_async(wr, L.ldx, p.router, E, D);
+  // ---- x and the router into shared memory; this CTA's share of every
+  // expert's weights into L2
+  stage_async(xs, L.ldx, p.x, D, T, D, vec);
+  stage_async(wr, L.ldx, p.router, D, E, D, vec);
   cp_async_commit();
-  stage_async(w1, L.ldw1, p.gu + static_cast<size_t>(me) * gu_rows * D, gu_rows, D);
-  stage_async(w2, L.ldw2, p.dn + static_cast<size_t>(me) * D * F, D, F);
-  cp_async_commit();
-  cp_async_wait<1>();
+  if (vec && warp == kWarps - 1) {
+    size_t lo, hi;
+    share_of(static_cast<size_t>(E) * gu_rows * D * sizeof(float), C, me, lo, hi);
+    if (lo < hi) prefetch_l2(p.gu, lo, hi, lane);
+    share_of(static_cast<size_t>(E) * D * F * sizeof(float), C, me, lo, hi);
+    if (lo < hi) prefetch_l2(p.dn, lo, hi, lane);
+  }
+  cp_async_wait_all();
   __syncthreads();
 
   // ---- router: logits of every (token, expert), four partial sums each
@@ -231,9 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
       }
     }
   }
-  // ---- each slot's row within its expert = the earlier tokens that chose
-  // the same expert (an expert's rows are listed in token order): per expert
-  // a warp ballot over the tokens, then the counts of the earlier warps
+  // ---- per expert and warp, how many of the warp's tokens chose it (one
+  // ballot per expert); a slot's row within its expert is the count of the
+  // earlier tokens that chose the same expert (rows listed in token order)
   int below[kSmallMaxExperts];
 #pragma unroll
   for (int e = 0; e < kSmallMaxExperts; ++e) {
@@ -242,8 +297,77 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
     if (lane == 0) wcnt[warp * kSmallMaxExperts + e] = __popc(b);
   }
   __syncthreads();
-  int rows = 0;                                // rows of expert `me`
-  for (int w = 0; w < kThreads / 32; ++w) rows += wcnt[w * kSmallMaxExperts + me];
+  // rows of every expert: lane e of each warp sums column e of the counts,
+  // then the warp shares the eight sums
+  int n[kSmallMaxExperts];
+  {
+    int mine = 0;
+    if (lane < kSmallMaxExperts)
+      for (int w = 0; w < kWarps; ++w) mine += wcnt[w * kSmallMaxExperts + lane];
+#pragma unroll
+    for (int e = 0; e < kSmallMaxExperts; ++e) {
+      const int v = __shfl_sync(0xffffffffu, mine, e);
+      n[e] = e < E ? v : 0;
+    }
+  }
+  // ---- the assignment of CTAs to (expert, slice), the same in every thread
+  // of every CTA: one CTA per expert with rows, then each further CTA to the
+  // expert with the most rows per CTA, while its columns still split into
+  // whole 4-column groups
+  const int groups4 = (F + 3) >> 2;
+  int s[kSmallMaxExperts];
+  int used = 0;
+#pragma unroll
+  for (int e = 0; e < kSmallMaxExperts; ++e) {
+    s[e] = n[e] > 0 ? 1 : 0;
+    used += s[e];
+  }
+  for (; used < C; ++used) {
+    int best = -1, bn = 0, bs = 1;
+#pragma unroll
+    for (int e = 0; e < kSmallMaxExperts; ++e)
+      if (s[e] > 0 && s[e] < groups4 && (best < 0 || n[e] * bs > bn * s[e])) {
+        best = e;
+        bn = n[e];
+        bs = s[e];
+      }
+    if (best < 0) break;
+#pragma unroll
+    for (int e = 0; e < kSmallMaxExperts; ++e) s[e] += e == best ? 1 : 0;
+  }
+  int my_e = -1, my_j = 0, my_s = 1, my_n = 0;
+  {
+    int cf = 0;
+#pragma unroll
+    for (int e = 0; e < kSmallMaxExperts; ++e) {
+      if (me >= cf && me < cf + s[e]) {
+        my_e = e;
+        my_j = me - cf;
+        my_s = s[e];
+        my_n = n[e];
+      }
+      if (tid == 0) {
+        cfirst[e] = cf;
+        scount[e] = s[e];
+      }
+      cf += s[e];
+    }
+  }
+  // this CTA's columns [f0, f1): slices of whole 4-column groups (a CTA
+  // left over when every expert is split to single groups has none)
+  const int f0 = my_e >= 0 ? 4 * (groups4 * my_j / my_s) : 0;
+  const int f1 = my_e >= 0 ? min(F, 4 * (groups4 * (my_j + 1) / my_s)) : 0;
+  const int wdt = f1 - f0;
+  const int ld2 = ld_odd4(wdt);
+  // ---- stage the slice's weights while the rows are listed
+  if (my_e >= 0) {
+    const float* gu_e = p.gu + static_cast<size_t>(my_e) * gu_rows * D;
+    stage_async(w1, L.ldx, gu_e + static_cast<size_t>(f0) * D, D, wdt, D, vec);
+    if (kGated)
+      stage_async(w1 + wdt * L.ldx, L.ldx, gu_e + static_cast<size_t>(F + f0) * D, D, wdt, D, vec);
+    stage_async(w2, ld2, p.dn + static_cast<size_t>(my_e) * D * F + f0, F, D, wdt, vec);
+  }
+  cp_async_commit();
   if (t < T) {
     for (int k = 0; k < K; ++k) {
       const int e = sel[t * K + k];
@@ -253,53 +377,48 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
         if (ee == e) r = below[ee];
       for (int w = 0; w < warp; ++w) r += wcnt[w * kSmallMaxExperts + e];
       rank[t * K + k] = r;
-      if (e == me) tok[r] = t;
+      if (e == my_e) tok[r] = t;
     }
   }
-  cp_async_wait<0>();
+  cp_async_wait_all();
   __syncthreads();
 
-  // ---- expert `me` on its rows: H, then Y (fp32 FMA from shared memory)
+  const int rows = my_n;
   const int groups = (rows + kRowGroup - 1) / kRowGroup;
-  for (int item = tid; item < F * groups; item += kThreads) {
-    const int f = item % F, g = item / F;
+  const int ldh = round4(wdt);
+  // ---- H[:, f0:f1] of expert my_e on its rows (fp32 FMA from shared memory)
+  for (int item = tid; item < wdt * groups; item += kThreads) {
+    const int f = item % wdt, g = item / wdt;
     float a[kRowGroup], b[kRowGroup];
 #pragma unroll
     for (int j = 0; j < kRowGroup; ++j) a[j] = b[j] = 0.f;
-    const float* wa = w1 + f * L.ldw1;                         // gate row (or W1 row)
-    const float* wb = w1 + (kGated ? F + f : f) * L.ldw1;     // up row
+    const float* wa = w1 + f * L.ldx;                          // gate row (or W1 row)
+    const float* wb = w1 + (kGated ? wdt + f : f) * L.ldx;     // up row
     const float* xr[kRowGroup];
 #pragma unroll
     for (int j = 0; j < kRowGroup; ++j) {
       const int r = g * kRowGroup + j;
       xr[j] = xs + (r < rows ? tok[r] : 0) * L.ldx;
     }
-    // x rows four columns at a time (16-byte reads every lane shares)
     int d = 0;
 #pragma unroll 2
     for (; d + 4 <= D; d += 4) {
       float4 xv[kRowGroup];
 #pragma unroll
       for (int j = 0; j < kRowGroup; ++j) xv[j] = *reinterpret_cast<const float4*>(xr[j] + d);
-      const float va[4] = {wa[d], wa[d + 1], wa[d + 2], wa[d + 3]};
-      float vb[4] = {0.f, 0.f, 0.f, 0.f};
-      if (kGated) {
-        vb[0] = wb[d];
-        vb[1] = wb[d + 1];
-        vb[2] = wb[d + 2];
-        vb[3] = wb[d + 3];
-      }
+      const float4 va = *reinterpret_cast<const float4*>(wa + d);
+      const float4 vb = kGated ? *reinterpret_cast<const float4*>(wb + d) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int j = 0; j < kRowGroup; ++j) {
-        a[j] = fmaf(xv[j].x, va[0], a[j]);
-        a[j] = fmaf(xv[j].y, va[1], a[j]);
-        a[j] = fmaf(xv[j].z, va[2], a[j]);
-        a[j] = fmaf(xv[j].w, va[3], a[j]);
+        a[j] = fmaf(xv[j].x, va.x, a[j]);
+        a[j] = fmaf(xv[j].y, va.y, a[j]);
+        a[j] = fmaf(xv[j].z, va.z, a[j]);
+        a[j] = fmaf(xv[j].w, va.w, a[j]);
         if (kGated) {
-          b[j] = fmaf(xv[j].x, vb[0], b[j]);
-          b[j] = fmaf(xv[j].y, vb[1], b[j]);
-          b[j] = fmaf(xv[j].z, vb[2], b[j]);
-          b[j] = fmaf(xv[j].w, vb[3], b[j]);
+          b[j] = fmaf(xv[j].x, vb.x, b[j]);
+          b[j] = fmaf(xv[j].y, vb.y, b[j]);
+          b[j] = fmaf(xv[j].z, vb.z, b[j]);
+          b[j] = fmaf(xv[j].w, vb.w, b[j]);
         }
       }
     }
@@ -313,43 +432,44 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
         if (kGated) b[j] = fmaf(xv, vb, b[j]);
       }
     }
-    const float bias = (!kGated && p.b1) ? __ldg(p.b1 + static_cast<size_t>(me) * F + f) : 0.f;
+    const float bias = (!kGated && p.b1) ? __ldg(p.b1 + static_cast<size_t>(my_e) * F + f0 + f) : 0.f;
 #pragma unroll
     for (int j = 0; j < kRowGroup; ++j) {
       const int r = g * kRowGroup + j;
       if (r < rows)
-        hs[r * L.ldh + f] = kGated ? a[j] / (1.f + expf(-a[j])) * b[j] : fmaxf(a[j] + bias, 0.f);
+        hs[r * ldh + f] = kGated ? a[j] / (1.f + expf(-a[j])) * b[j] : fmaxf(a[j] + bias, 0.f);
     }
   }
   __syncthreads();
+  // ---- this slice's share of Y = H Wd^T (+ b2 once, in the first slice)
   for (int item = tid; item < D * groups; item += kThreads) {
     const int d = item % D, g = item / D;
     float a[kRowGroup];
 #pragma unroll
     for (int j = 0; j < kRowGroup; ++j) a[j] = 0.f;
-    const float* wd = w2 + d * L.ldw2;
+    const float* wd = w2 + d * ld2;
     const float* hr[kRowGroup];
 #pragma unroll
-    for (int j = 0; j < kRowGroup; ++j) hr[j] = hs + min(g * kRowGroup + j, rows - 1) * L.ldh;
+    for (int j = 0; j < kRowGroup; ++j) hr[j] = hs + min(g * kRowGroup + j, rows - 1) * ldh;
     int f = 0;
 #pragma unroll 2
-    for (; f + 4 <= F; f += 4) {
-      const float v[4] = {wd[f], wd[f + 1], wd[f + 2], wd[f + 3]};
+    for (; f + 4 <= wdt; f += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(wd + f);
 #pragma unroll
       for (int j = 0; j < kRowGroup; ++j) {
         const float4 h4 = *reinterpret_cast<const float4*>(hr[j] + f);
-        a[j] = fmaf(h4.x, v[0], a[j]);
-        a[j] = fmaf(h4.y, v[1], a[j]);
-        a[j] = fmaf(h4.z, v[2], a[j]);
-        a[j] = fmaf(h4.w, v[3], a[j]);
+        a[j] = fmaf(h4.x, v.x, a[j]);
+        a[j] = fmaf(h4.y, v.y, a[j]);
+        a[j] = fmaf(h4.z, v.z, a[j]);
+        a[j] = fmaf(h4.w, v.w, a[j]);
       }
     }
-    for (; f < F; ++f) {
+    for (; f < wdt; ++f) {
       const float v = wd[f];
 #pragma unroll
       for (int j = 0; j < kRowGroup; ++j) a[j] = fmaf(hr[j][f], v, a[j]);
     }
-    const float bias = p.b2 ? __ldg(p.b2 + static_cast<size_t>(me) * D + d) : 0.f;
+    const float bias = (p.b2 && my_j == 0) ? __ldg(p.b2 + static_cast<size_t>(my_e) * D + d) : 0.f;
 #pragma unroll
     for (int j = 0; j < kRowGroup; ++j) {
       const int r = g * kRowGroup + j;
@@ -357,15 +477,19 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
     }
   }
 
-  // ---- combine: every expert's rows are in its CTA's shared memory
+  // ---- combine: every slice's share of Y is in its CTA's shared memory
   cluster_barrier();
-  const int t_lo = me * T / E, t_hi = (me + 1) * T / E;
+  const int t_lo = me * T / C, t_hi = (me + 1) * T / C;
   for (int i = tid; i < (t_hi - t_lo) * D; i += kThreads) {
     const int tt = t_lo + i / D, d = i % D;
     float acc = 0.f;
     for (int k = 0; k < K; ++k) {
       const int e = sel[tt * K + k];
-      acc = fmaf(wsel[tt * K + k], ld_remote_f32(ys + rank[tt * K + k] * D + d, e), acc);
+      const float* yrow = ys + rank[tt * K + k] * D + d;
+      const int c0 = cfirst[e], ns = scount[e];
+      float y = 0.f;
+      for (int j = 0; j < ns; ++j) y += ld_remote_f32(yrow, static_cast<uint32_t>(c0 + j));
+      acc = fmaf(wsel[tt * K + k], y, acc);
     }
     p.out[static_cast<size_t>(tt) * D + d] = acc;
   }
@@ -375,6 +499,35 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
 
 size_t small_smem_bytes(int T, int D, int F, int E, int K, int gated) {
   return sizeof(float) * static_cast<size_t>(small_layout(T, D, F, E, K, gated).total);
+}
+
+// The automatic cluster size of a device: 16 CTAs when a cluster of 16 of
+// these CTAs (512 threads, the largest shared-memory size this kernel is
+// launched with) can be resident at once, else the portable 8.
+int auto_cluster(int dev) {
+  static std::mutex mu;
+  static int cached[64] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  int c = kSmallMinCluster;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kSmallMaxCluster);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmallMaxSmem;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = kSmallMaxCluster;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int nclusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&nclusters, small_layer_f32_kernel<true>, &cfg) == cudaSuccess &&
+      nclusters >= 1)
+    c = kSmallMaxCluster;
+  (void)cudaGetLastError();   // a refused query leaves no error behind
+  if (dev >= 0 && dev < 64) cached[dev] = c;
+  return c;
 }
 
 }  // namespace
@@ -389,8 +542,10 @@ cudaError_t launch_small_layer_f32(const float* x, const float* router, const fl
                                    const float* gu, const float* dn, const float* b1,
                                    const float* b2, int T, int D, int F, int E, int K, int norm,
                                    int gated, float* out, int64_t* sel64, float* wout,
-                                   float* logits, cudaStream_t s) {
+                                   float* logits, int cluster, cudaStream_t s) {
   if (!small_layer_fits(T, D, F, E, K, gated)) return cudaErrorInvalidValue;
+  if (cluster != 0 && cluster != kSmallMinCluster && cluster != kSmallMaxCluster)
+    return cudaErrorInvalidValue;
   static std::mutex mu;
   static bool done[64] = {};
   int dev = 0;
@@ -403,10 +558,13 @@ cudaError_t launch_small_layer_f32(const float* x, const float* router, const fl
         err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    static_cast<int>(kSmallMaxSmem));
         if (err != cudaSuccess) return err;
+        err = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (err != cudaSuccess) return err;
       }
       if (dev >= 0 && dev < 64) done[dev] = true;
     }
   }
+  const int C = cluster ? cluster : auto_cluster(dev);
   SmallParams p;
   p.x = x;
   p.router = router;
@@ -425,9 +583,10 @@ cudaError_t launch_small_layer_f32(const float* x, const float* router, const fl
   p.E = E;
   p.K = K;
   p.norm = norm;
-  p.gated = gated;
-  return launch_k(gated ? small_layer_f32_kernel<true> : small_layer_f32_kernel<false>, dim3(E),
-                  dim3(kThreads), small_smem_bytes(T, D, F, E, K, gated), s, pdl_enabled(), E, p);
+  p.C = C;
+  p.vec = (D % 4 == 0 && F % 4 == 0) ? 1 : 0;
+  return launch_k(gated ? small_layer_f32_kernel<true> : small_layer_f32_kernel<false>, dim3(C),
+                  dim3(kThreads), small_smem_bytes(T, D, F, E, K, gated), s, pdl_enabled(), C, p);
 }
 
 }  // namespace moe

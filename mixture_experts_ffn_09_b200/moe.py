@@ -123,6 +123,8 @@ def lib() -> ctypes.CDLL:
         L.moe_set_fused_gather.restype = i32
         L.moe_set_gemm_mode.argtypes = [i32]
         L.moe_set_gemm_mode.restype = i32
+        L.moe_set_small_cluster.argtypes = [i32]
+        L.moe_set_small_cluster.restype = i32
         L.moe_stage_name.argtypes = [i32]
         L.moe_stage_name.restype = ctypes.c_char_p
         _lib = L
@@ -394,6 +396,18 @@ def set_tail_swap(max_rows: int) -> int:
     prev = int(lib().moe_set_tail_swap(int(max_rows)))
     if prev < 0:
         raise ValueError(f"tail swap rows out of range: {max_rows}")
+    return prev
+
+
+SMALL_CLUSTER_AUTO = 0
+
+
+def set_small_cluster(ctas: int) -> int:
+    """Cluster size of the one-kernel float32 small layer: SMALL_CLUSTER_AUTO
+    (16 where possible, else 8), 8 or 16.  Returns the previous value."""
+    prev = int(lib().moe_set_small_cluster(int(ctas)))
+    if prev < 0:
+        raise ValueError(f"small-layer cluster size must be 0, 8 or 16, not {ctas}")
     return prev
 
 

@@ -73,6 +73,17 @@ def test_process_wide_settings_validate_on_host(L):
         assert L.moe_set_gemm_mode(1) == 2
     finally:
         L.moe_set_gemm_mode(g)
+    c = L.moe_set_small_cluster(8)
+    try:
+        assert c == 0                              # MOE_SMALL_CLUSTER_AUTO
+        for bad in (1, 4, 12, 32, -1):
+            assert L.moe_set_small_cluster(bad) == -1
+        assert L.moe_set_small_cluster(16) == 8
+        with pytest.raises(ValueError):
+            moe.set_small_cluster(9)
+        assert moe.set_small_cluster(moe.SMALL_CLUSTER_AUTO) == 16
+    finally:
+        L.moe_set_small_cluster(c)
 
 
 C_CALLER = r'''

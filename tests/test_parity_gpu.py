@@ -530,6 +530,51 @@ def test_small_float32_layer_runs_as_one_kernel(name):
     PL.check_out(res[0]["out"][same], res[1]["out"][same], "f32", "one kernel vs six")
 
 
+def _skewed_small(seed, T, D, F, E, act, hot):
+    """A small fp32 case whose router sends every token's first choice to
+    expert `hot` (a large router bias), the rest by the logits."""
+    d = dict(synth.random_case(seed, T, D, F, E, act=act, dtype="f32", weight_std=0.3))
+    rb = np.zeros(E, dtype=np.float32) if d["router_bias"] is None else d["router_bias"].copy()
+    rb[hot] += np.float32(40.0)
+    d["router_bias"] = rb
+    return d
+
+
+SMALL_SPLIT_CASES = [
+    # (seed, T, D, F, E, K, act, skew)
+    (61, 64, 64, 128, 8, 2, "silu_gated", True),     # one expert takes every token
+    (62, 64, 32, 64, 4, 2, "relu", True),
+    (63, 1, 64, 128, 8, 2, "silu_gated", False),     # a single token
+    (64, 32, 16, 32, 8, 8, "silu_gated", False),     # K = E: every expert, T*K = 256
+    (65, 256, 16, 24, 3, 1, "relu", True),           # T*K = 256 on one expert
+    (66, 40, 33, 47, 5, 2, "silu_gated", False),     # D, F not multiples of 4: 4-byte copies
+    (67, 50, 8, 4, 2, 1, "silu_gated", True),        # F = 4: one column group, no split
+    (68, 20, 12, 10, 1, 1, "relu", False),           # E = 1
+]
+
+
+@pytest.mark.parametrize("cluster", [8, 16])
+@pytest.mark.parametrize("seed,T,D,F,E,K,act,skew", SMALL_SPLIT_CASES)
+def test_small_layer_split_over_the_cluster(seed, T, D, F, E, K, act, skew, cluster):
+    """The one-kernel small layer splits each expert's hidden columns over
+    CTAs in proportion to its rows.  Skewed routing (one expert with every
+    token), a single token, K = E, column counts that do not split into
+    4-column groups evenly or at all, and one expert: every token against
+    the oracle, with clusters of 8 and of 16 CTAs, in one launch each."""
+    from mixture_experts_ffn_09_b200 import moe
+    d = _skewed_small(seed, T, D, F, E, act, seed % E) if skew else \
+        synth.random_case(seed, T, D, F, E, act=act, dtype="f32", weight_std=0.3)
+    prev = moe.set_small_cluster(cluster)
+    try:
+        n0 = moe.kernel_launches()
+        g, _ = _full_check(d, E, K, True, act, "f32")
+        assert moe.kernel_launches() - n0 == 1
+    finally:
+        moe.set_small_cluster(prev)
+    if skew:
+        assert (g["sel"][:, 0] == seed % E).all()
+
+
 @pytest.mark.parametrize("act", ["silu_gated", "relu"])
 def test_split_last_wave(act):
     """Layers in the CTA-pair regime run their last wave as k-halves: the
