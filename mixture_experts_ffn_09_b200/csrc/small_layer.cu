@@ -50,6 +50,9 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRowGroup = 4;      // rows of one expert computed together by a thread
+constexpr int kLogitT = 2;        // router: tokens ...
+constexpr int kLogitE = 4;        // ... x experts computed together by a thread
+constexpr int kSplit = 8;         // router: lanes that split D for one (tokens, experts) block
 
 struct SmallParams {
   const float* x;
@@ -81,9 +84,13 @@ __host__ __device__ constexpr int ld_odd4(int v) {
 // The weight, H and Y regions are sized for the largest case: one slice of
 // all F columns, an expert chosen by all T tokens.
 struct SmallLayout {
-  int xs, wr, lg, sel, w, rank, tok, wcnt, cfirst, scount, w1, w2, h, y, total;
+  int xs, wr, rbs, lg, sel, w, rank, tok, wcnt, cnt, cfirst, scount, w1, w2, b1s, b2s, h, y, total;
   int ldx;    // rows of x, of the router and of the staged gate/up weights
 };
+
+// Row counts are kept per group of 4 tokens (the tokens of one warp in the
+// top-k, 8 lanes per token).
+__host__ __device__ constexpr int token_quads(int T) { return (T + 3) / 4; }
 
 __host__ __device__ inline SmallLayout small_layout(int T, int D, int F, int E, int K, int gated) {
   SmallLayout L;
@@ -92,16 +99,20 @@ __host__ __device__ inline SmallLayout small_layout(int T, int D, int F, int E, 
   int o = 0;
   L.xs = o;     o += round4(T * L.ldx);
   L.wr = o;     o += round4(E * L.ldx);
+  L.rbs = o;    o += kSmallMaxExperts;
   L.lg = o;     o += round4(T * E);
   L.sel = o;    o += round4(T * K);
   L.w = o;      o += round4(T * K);
   L.rank = o;   o += round4(T * K);
   L.tok = o;    o += round4(T);
-  L.wcnt = o;   o += kWarps * kSmallMaxExperts;
+  L.wcnt = o;   o += token_quads(T) * kSmallMaxExperts;
+  L.cnt = o;    o += kSmallMaxExperts;
   L.cfirst = o; o += kSmallMaxExperts;
   L.scount = o; o += kSmallMaxExperts;
   L.w1 = o;     o += (gated ? 2 : 1) * fmax * L.ldx;
   L.w2 = o;     o += D * ld_odd4(F);
+  L.b1s = o;    o += fmax;
+  L.b2s = o;    o += round4(D);
   L.h = o;      o += T * fmax;
   L.y = o;      o += round4(T * D);
   L.total = o;
@@ -194,28 +205,34 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
   const SmallLayout L = small_layout(T, D, F, E, K, kGated);
   float* xs = sm + L.xs;
   float* wr = sm + L.wr;
+  float* rbs = sm + L.rbs;
   float* lg = sm + L.lg;
   int* sel = reinterpret_cast<int*>(sm + L.sel);
   float* wsel = sm + L.w;
   int* rank = reinterpret_cast<int*>(sm + L.rank);
   int* tok = reinterpret_cast<int*>(sm + L.tok);
   int* wcnt = reinterpret_cast<int*>(sm + L.wcnt);
+  int* cnt = reinterpret_cast<int*>(sm + L.cnt);
   int* cfirst = reinterpret_cast<int*>(sm + L.cfirst);
   int* scount = reinterpret_cast<int*>(sm + L.scount);
   float* w1 = sm + L.w1;
   float* w2 = sm + L.w2;
+  float* b1s = sm + L.b1s;
+  float* b2s = sm + L.b2s;
   float* hs = sm + L.h;
   float* ys = sm + L.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const unsigned full = 0xffffffffu;
   const int me = static_cast<int>(cta_rank());
   const int gu_rows = kGated ? 2 * F : F;
 
   pdl_trigger();
   pdl_wait();
-  // ---- x and the router into shared memory; this CTA's share of every
-  // expert's weights into L2
+  // ---- x, the router and its bias into shared memory; this CTA's share of
+  // every expert's weights into L2
   stage_async(xs, L.ldx, p.x, D, T, D, vec);
   stage_async(wr, L.ldx, p.router, D, E, D, vec);
+  if (p.rb) stage_async(rbs, E, p.rb, E, 1, E, false);
   cp_async_commit();
   if (vec && warp == kWarps - 1) {
     size_t lo, hi;
@@ -227,130 +244,187 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
   cp_async_wait_all();
   __syncthreads();
 
-  // ---- router: logits of every (token, expert), four partial sums each
-  for (int i = tid; i < T * E; i += kThreads) {
-    const int t = i / E, e = i % E;
-    const float* xr = xs + t * L.ldx;
-    const float* rr = wr + e * L.ldx;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    int d = 0;
-    for (; d + 4 <= D; d += 4) {
-      const float4 xv = *reinterpret_cast<const float4*>(xr + d);
-      const float4 rv = *reinterpret_cast<const float4*>(rr + d);
-      a0 = fmaf(xv.x, rv.x, a0);
-      a1 = fmaf(xv.y, rv.y, a1);
-      a2 = fmaf(xv.z, rv.z, a2);
-      a3 = fmaf(xv.w, rv.w, a3);
+  // ---- router: logits of every (token, expert).  Eight consecutive lanes
+  // share 2 tokens x 4 experts and split D between them (lane c takes the
+  // 4-float chunks c, c + 8, ...), so every x and router value a lane reads
+  // feeds 4 or 2 FMAs; the eight partial sums are added by a butterfly of
+  // shuffles.  Every CTA runs the same code on the same data.
+  {
+    const int nq = (E + kLogitE - 1) / kLogitE;
+    const int items = ((T + kLogitT - 1) / kLogitT) * nq;
+    const int c = lane & (kSplit - 1);
+    for (int it = 0; it < (items + kThreads / kSplit - 1) / (kThreads / kSplit); ++it) {
+      const int item = it * (kThreads / kSplit) + tid / kSplit;    // the same in all 8 lanes
+      const bool ok = item < items;
+      const int t0 = ok ? (item / nq) * kLogitT : 0, e0 = ok ? (item % nq) * kLogitE : 0;
+      const float* xr[kLogitT];
+      const float* rr[kLogitE];
+#pragma unroll
+      for (int u = 0; u < kLogitT; ++u) xr[u] = xs + min(t0 + u, T - 1) * L.ldx;
+#pragma unroll
+      for (int v = 0; v < kLogitE; ++v) rr[v] = wr + min(e0 + v, E - 1) * L.ldx;
+      float a[kLogitT][kLogitE];
+#pragma unroll
+      for (int u = 0; u < kLogitT; ++u)
+#pragma unroll
+        for (int v = 0; v < kLogitE; ++v) a[u][v] = 0.f;
+      if (ok) {
+        int d = 4 * c;
+        for (; d + 4 <= D; d += 4 * kSplit) {
+          float4 xv[kLogitT];
+#pragma unroll
+          for (int u = 0; u < kLogitT; ++u) xv[u] = *reinterpret_cast<const float4*>(xr[u] + d);
+#pragma unroll
+          for (int v = 0; v < kLogitE; ++v) {
+            const float4 rv = *reinterpret_cast<const float4*>(rr[v] + d);
+#pragma unroll
+            for (int u = 0; u < kLogitT; ++u) {
+              a[u][v] = fmaf(xv[u].x, rv.x, a[u][v]);
+              a[u][v] = fmaf(xv[u].y, rv.y, a[u][v]);
+              a[u][v] = fmaf(xv[u].z, rv.z, a[u][v]);
+              a[u][v] = fmaf(xv[u].w, rv.w, a[u][v]);
+            }
+          }
+        }
+        // D not a multiple of 4: the last D % 4 columns, in the lane whose
+        // next chunk would have held them
+        if (d < D && d + 4 > D)
+          for (; d < D; ++d)
+#pragma unroll
+            for (int u = 0; u < kLogitT; ++u)
+#pragma unroll
+              for (int v = 0; v < kLogitE; ++v) a[u][v] = fmaf(xr[u][d], rr[v][d], a[u][v]);
+      }
+#pragma unroll
+      for (int o = 1; o < kSplit; o <<= 1)
+#pragma unroll
+        for (int u = 0; u < kLogitT; ++u)
+#pragma unroll
+          for (int v = 0; v < kLogitE; ++v) a[u][v] += __shfl_xor_sync(full, a[u][v], o);
+      if (ok && c == 0) {
+#pragma unroll
+        for (int u = 0; u < kLogitT; ++u)
+#pragma unroll
+          for (int v = 0; v < kLogitE; ++v) {
+            const int t = t0 + u, e = e0 + v;
+            if (t < T && e < E) {
+              const float acc = p.rb ? a[u][v] + rbs[e] : a[u][v];
+              lg[t * E + e] = acc;
+              if (me == 0 && p.logits) p.logits[t * E + e] = acc;
+            }
+          }
+      }
     }
-    for (; d < D; ++d) a0 = fmaf(xr[d], rr[d], a0);
-    float acc = (a0 + a1) + (a2 + a3);
-    if (p.rb) acc += __ldg(p.rb + e);
-    lg[i] = acc;
-    if (me == 0 && p.logits) p.logits[i] = acc;
   }
   __syncthreads();
-  // ---- softmax, top-k and weights, one thread per token (T <= kThreads)
-  const int t = tid;
-  unsigned int member = 0u;                    // experts token t chose
-  if (t < T) {
-    const float* l = lg + t * E;
-    float m = -INFINITY;
-    for (int e = 0; e < E; ++e) m = fmaxf(m, isnan(l[e]) ? -INFINITY : l[e]);
-    float s = 0.f;
-    for (int e = 0; e < E; ++e) s += isnan(l[e]) ? 0.f : expf(l[e] - m);
-    // the K best by logit (softmax is monotone), a NaN logit ranking last
-    float psum = 0.f;
-    for (int k = 0; k < K; ++k) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
-      for (int e = 0; e < E; ++e) {
-        const float v = isnan(l[e]) ? -INFINITY : l[e];
-        if (!(member & (1u << e)) && ranks_before(v, e, bv, be)) {
-          bv = v;
-          be = e;
-        }
-      }
-      member |= 1u << be;
-      const float pk = isnan(l[be]) ? 0.f : expf(l[be] - m) / s;
-      sel[t * K + k] = be;
-      wsel[t * K + k] = pk;
-      psum += pk;
+
+  // ---- softmax, top-k and weights: eight lanes per token, lane e holding
+  // expert e (lanes e >= E hold nothing and rank after every expert).  The
+  // K best by logit (softmax is monotone; a NaN logit ranks last, equal
+  // logits to the lower index) are the lanes with fewer than K lanes ranking
+  // before them; lane rank k writes slot k.  One ballot per warp then gives,
+  // for each selected slot, the earlier tokens of the warp that chose the
+  // same expert, and per expert the count of the warp's 4 tokens.
+  for (int it = 0; it < (T + kThreads / 8 - 1) / (kThreads / 8); ++it) {
+    const int t = it * (kThreads / 8) + tid / 8, e = lane & 7;
+    const bool valid = t < T && e < E;
+    const float l = valid ? lg[t * E + e] : NAN;
+    const float v = isnan(l) ? -INFINITY : l;
+    float m = v;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(full, m, o));
+    const float ex = (valid && !isnan(l)) ? expf(l - m) : 0.f;
+    float s = ex;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) s += __shfl_xor_sync(full, s, o);
+    int k = 0;                                 // lanes of this token ranking before e
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float vj = __shfl_sync(full, v, (lane & ~7) | j);
+      k += ranks_before(vj, j, v, e) ? 1 : 0;
     }
-    const float denom = psum + 1e-9f;
-    for (int k = 0; k < K; ++k) {
-      const float w = p.norm ? wsel[t * K + k] / denom : wsel[t * K + k];
+    const bool chosen = valid && k < K;
+    const float pk = chosen ? (isnan(l) ? 0.f : ex / s) : 0.f;
+    float psum = pk;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) psum += __shfl_xor_sync(full, psum, o);
+    const unsigned int b = __ballot_sync(full, chosen);
+    const unsigned int col = 0x01010101u << e;     // expert e's lane in each of the 4 tokens
+    if (chosen) {
+      const float w = p.norm ? pk / (psum + 1e-9f) : pk;
+      sel[t * K + k] = e;
       wsel[t * K + k] = w;
+      rank[t * K + k] = __popc(b & col & lanemask_lt());   // completed below
       if (me == 0) {
-        if (p.sel64) p.sel64[static_cast<size_t>(t) * K + k] = sel[t * K + k];
+        if (p.sel64) p.sel64[static_cast<size_t>(t) * K + k] = e;
         if (p.wout) p.wout[static_cast<size_t>(t) * K + k] = w;
       }
     }
-  }
-  // ---- per expert and warp, how many of the warp's tokens chose it (one
-  // ballot per expert); a slot's row within its expert is the count of the
-  // earlier tokens that chose the same expert (rows listed in token order)
-  int below[kSmallMaxExperts];
-#pragma unroll
-  for (int e = 0; e < kSmallMaxExperts; ++e) {
-    const unsigned int b = __ballot_sync(0xffffffffu, (member >> e) & 1u);
-    below[e] = __popc(b & lanemask_lt());
-    if (lane == 0) wcnt[warp * kSmallMaxExperts + e] = __popc(b);
+    const int quad = it * (kThreads / 32) + warp;
+    if (lane < 8 && quad < token_quads(T)) wcnt[quad * kSmallMaxExperts + lane] = __popc(b & col);
   }
   __syncthreads();
-  // rows of every expert: lane e of each warp sums column e of the counts,
-  // then the warp shares the eight sums
-  int n[kSmallMaxExperts];
-  {
-    int mine = 0;
-    if (lane < kSmallMaxExperts)
-      for (int w = 0; w < kWarps; ++w) mine += wcnt[w * kSmallMaxExperts + lane];
+  // ---- per expert (warp e), the exclusive prefix of the quads' counts, in
+  // place, and the expert's total rows
+  if (warp < E) {
+    const int e = warp, nquads = token_quads(T);
+    int total = 0;
+    for (int q0 = 0; q0 < nquads; q0 += 32) {
+      const int q = q0 + lane;
+      const int c0 = q < nquads ? wcnt[q * kSmallMaxExperts + e] : 0;
+      int inc = c0;
 #pragma unroll
-    for (int e = 0; e < kSmallMaxExperts; ++e) {
-      const int v = __shfl_sync(0xffffffffu, mine, e);
-      n[e] = e < E ? v : 0;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(full, inc, o);
+        if (lane >= o) inc += y;
+      }
+      if (q < nquads) wcnt[q * kSmallMaxExperts + e] = total + inc - c0;
+      total += __shfl_sync(full, inc, 31);
     }
+    if (lane == 0) cnt[e] = total;
   }
-  // ---- the assignment of CTAs to (expert, slice), the same in every thread
-  // of every CTA: one CTA per expert with rows, then each further CTA to the
-  // expert with the most rows per CTA, while its columns still split into
-  // whole 4-column groups
+  __syncthreads();
+  // ---- the assignment of CTAs to (expert, slice), computed by every warp
+  // with lane e standing for expert e, so all threads of all CTAs agree.
+  // Each expert with rows gets one CTA plus its proportional share of the
+  // other C - A (rounded down; at most one CTA per 4-column group of F);
+  // each CTA still free then goes to the expert with the most rows per CTA
+  // (lower index on ties) that can still be split.  The comparison uses
+  // n * 65536 / s, exact for these sizes: two different ratios n/s with
+  // s <= 16 differ by at least 1/256.
   const int groups4 = (F + 3) >> 2;
-  int s[kSmallMaxExperts];
-  int used = 0;
-#pragma unroll
-  for (int e = 0; e < kSmallMaxExperts; ++e) {
-    s[e] = n[e] > 0 ? 1 : 0;
-    used += s[e];
-  }
-  for (; used < C; ++used) {
-    int best = -1, bn = 0, bs = 1;
-#pragma unroll
-    for (int e = 0; e < kSmallMaxExperts; ++e)
-      if (s[e] > 0 && s[e] < groups4 && (best < 0 || n[e] * bs > bn * s[e])) {
-        best = e;
-        bn = n[e];
-        bs = s[e];
-      }
-    if (best < 0) break;
-#pragma unroll
-    for (int e = 0; e < kSmallMaxExperts; ++e) s[e] += e == best ? 1 : 0;
-  }
-  int my_e = -1, my_j = 0, my_s = 1, my_n = 0;
+  int my_e, my_j, my_s, my_n;
   {
-    int cf = 0;
+    const int ne = lane < E ? cnt[lane] : 0;
+    const int R = __reduce_add_sync(full, ne);
+    const int A = __popc(__ballot_sync(full, ne > 0));
+    int se = ne > 0 ? 1 + min(groups4 - 1, ne * (C - A) / R) : 0;
+    for (int used = __reduce_add_sync(full, se); used < C; ++used) {
+      const bool can = se > 0 && se < groups4;
+      const unsigned int key =
+          can ? (((static_cast<unsigned int>(ne) << 16) / static_cast<unsigned int>(se)) << 3) |
+                    static_cast<unsigned int>(7 - lane)
+              : 0u;
+      const unsigned int best = __reduce_max_sync(full, key);
+      if (best == 0u) break;
+      if (lane == 7 - static_cast<int>(best & 7u)) ++se;
+    }
+    int cf = se;                               // inclusive scan over the experts
 #pragma unroll
-    for (int e = 0; e < kSmallMaxExperts; ++e) {
-      if (me >= cf && me < cf + s[e]) {
-        my_e = e;
-        my_j = me - cf;
-        my_s = s[e];
-        my_n = n[e];
-      }
-      if (tid == 0) {
-        cfirst[e] = cf;
-        scount[e] = s[e];
-      }
-      cf += s[e];
+    for (int o = 1; o < 8; o <<= 1) {
+      const int y = __shfl_up_sync(full, cf, o);
+      if (lane >= o) cf += y;
+    }
+    cf -= se;
+    const unsigned int hit = __ballot_sync(full, lane < 8 && se > 0 && me >= cf && me < cf + se);
+    my_e = hit ? __ffs(hit) - 1 : -1;
+    const int src = my_e >= 0 ? my_e : 0;
+    my_j = me - __shfl_sync(full, cf, src);
+    my_s = __shfl_sync(full, se, src);
+    my_n = __shfl_sync(full, ne, src);
+    if (tid < kSmallMaxExperts) {
+      cfirst[tid] = cf;
+      scount[tid] = se;
     }
   }
   // this CTA's columns [f0, f1): slices of whole 4-column groups (a CTA
@@ -359,26 +433,24 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
   const int f1 = my_e >= 0 ? min(F, 4 * (groups4 * (my_j + 1) / my_s)) : 0;
   const int wdt = f1 - f0;
   const int ld2 = ld_odd4(wdt);
-  // ---- stage the slice's weights while the rows are listed
+  // ---- stage the slice's weights and biases while the rows are listed
   if (my_e >= 0) {
     const float* gu_e = p.gu + static_cast<size_t>(my_e) * gu_rows * D;
     stage_async(w1, L.ldx, gu_e + static_cast<size_t>(f0) * D, D, wdt, D, vec);
     if (kGated)
       stage_async(w1 + wdt * L.ldx, L.ldx, gu_e + static_cast<size_t>(F + f0) * D, D, wdt, D, vec);
     stage_async(w2, ld2, p.dn + static_cast<size_t>(my_e) * D * F + f0, F, D, wdt, vec);
+    if (!kGated && p.b1) stage_async(b1s, wdt, p.b1 + static_cast<size_t>(my_e) * F + f0, wdt, 1, wdt, vec);
+    if (p.b2 && my_j == 0) stage_async(b2s, D, p.b2 + static_cast<size_t>(my_e) * D, D, 1, D, vec);
   }
   cp_async_commit();
-  if (t < T) {
-    for (int k = 0; k < K; ++k) {
-      const int e = sel[t * K + k];
-      int r = 0;
-#pragma unroll
-      for (int ee = 0; ee < kSmallMaxExperts; ++ee)
-        if (ee == e) r = below[ee];
-      for (int w = 0; w < warp; ++w) r += wcnt[w * kSmallMaxExperts + e];
-      rank[t * K + k] = r;
-      if (e == my_e) tok[r] = t;
-    }
+  // each slot's row within its expert: earlier tokens of its warp (above)
+  // plus the expert's rows in earlier quads
+  for (int i = tid; i < T * K; i += kThreads) {
+    const int t = i / K, e = sel[i];
+    const int r = rank[i] + wcnt[(t >> 2) * kSmallMaxExperts + e];
+    rank[i] = r;
+    if (e == my_e) tok[r] = t;
   }
   cp_async_wait_all();
   __syncthreads();
@@ -432,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
         if (kGated) b[j] = fmaf(xv, vb, b[j]);
       }
     }
-    const float bias = (!kGated && p.b1) ? __ldg(p.b1 + static_cast<size_t>(my_e) * F + f0 + f) : 0.f;
+    const float bias = (!kGated && p.b1) ? b1s[f] : 0.f;
 #pragma unroll
     for (int j = 0; j < kRowGroup; ++j) {
       const int r = g * kRowGroup + j;
@@ -469,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1) small_layer_f32_kernel(const Smal
 #pragma unroll
       for (int j = 0; j < kRowGroup; ++j) a[j] = fmaf(hr[j][f], v, a[j]);
     }
-    const float bias = (p.b2 && my_j == 0) ? __ldg(p.b2 + static_cast<size_t>(my_e) * D + d) : 0.f;
+    const float bias = (p.b2 && my_j == 0) ? b2s[d] : 0.f;
 #pragma unroll
     for (int j = 0; j < kRowGroup; ++j) {
       const int r = g * kRowGroup + j;
