@@ -430,6 +430,46 @@ def time_steps(layer, steps, wd, world, local, what):
     return t0.elapsed_time(t1), launches, clk
 
 
+def time_graph_steps(layer, steps, wd, world, what):
+    """Device time of `steps` replays of one forward captured in a CUDA graph
+    (the same C-ABI call, recorded once after the warm-up), back to back on
+    the launching stream: the forward without the host's per-call work
+    (argument checks in the binding, the library's host side, the launch).
+    Returns ms of this rank over all replays."""
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    cap = torch.cuda.Stream(layer.dev)
+    cap.wait_stream(layer.stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        main = layer.stream
+        layer.stream = cap
+        try:
+            with torch.cuda.graph(g, stream=cap):
+                layer.step()
+        finally:
+            layer.stream = main
+    layer.stream.wait_stream(cap)
+    for _ in range(3):
+        g.replay()
+    wd.sync(f"before {what}")
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(layer.stream)
+    for _ in range(steps):
+        g.replay()
+    t1.record(layer.stream)
+    wd.sync(what)
+    ms = t0.elapsed_time(t1)
+    del g
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    return ms
+
+
 def stage_pass(layer, n, wd, local, what):
     """Per-stage CUDA-event times of n forwards (events between the kernels
     on the launching stream, so not the headline number), with the clocks
@@ -541,13 +581,20 @@ def measure_extra(w, args, dev, local, world, peaks):
     steps = max(5, min(args.steps, args.extra_steps))
     local_ms, launches, clk = time_steps(layer, steps, wd, world, local, f"{w.name} timed region")
     ms_step, tok_s = throughput(local_ms, steps, w.T, world, dev)
+    # replays: at least ~50 ms of them (thousands for the microsecond-scale layers)
+    g_steps = int(min(5000, max(steps, 50.0 / max(ms_step, 1e-3))))
+    g_ms, g_tok_s = throughput(time_graph_steps(layer, g_steps, wd, world, f"{w.name} graph replays"),
+                               g_steps, w.T, world, dev)
     per_call, sclk = stage_pass(layer, max(5, min(steps, 50)), wd, local, f"{w.name} per-stage pass")
     rflops = routed_flops(w)
     abytes = algorithmic_bytes(w, touched)
     r = {"config": workload_config(w, world), "steps": steps, "ms_per_step": round(ms_step, 4),
          "tokens_per_s": round(tok_s, 1), "routed_tflops": round(world * rflops / (ms_step / 1e3) / 1e12, 3),
          "stages_ms": {k: round(v, 4) for k, v in per_call.items()}, "gpu_launches": launches,
-         "experts_touched": touched, "clocks": clk}
+         "experts_touched": touched, "clocks": clk,
+         "graph": {"ms_per_step": round(g_ms, 4), "tokens_per_s": round(g_tok_s, 1), "replays": g_steps,
+                   "how": "the same forward captured once in a CUDA graph and replayed back to back "
+                          "(no per-call host work); ms_per_step above is the direct C-ABI call"}}
     if w.dtype == "bf16":
         r["roofline"] = gate_up_roofline(w, per_call, touched, peaks, args.gemm, local_ms / 1e3, sclk)
         if w.T * w.K <= 512:

@@ -453,6 +453,45 @@ def test_forward_replays_from_a_cuda_graph(gemm_mode):
     assert moe.device_status() == moe.MOE_OK
 
 
+@pytest.mark.parametrize("name", [synth.DENSE_RELU.name, synth.SILU_SMALL.name])
+def test_small_layer_replays_from_a_cuda_graph(name):
+    """The one-kernel small layer, captured once after a first call (which
+    sets the kernel attributes and picks the cluster size), replays from a
+    CUDA graph with the eager result bit for bit."""
+    import torch
+    from mixture_experts_ffn_09_b200 import moe
+    w = synth.WORKLOADS[name]
+    dev = PL.to_device(synth.make_inputs(w))
+    x = dev["x"].reshape(w.T, w.D)
+    a = moe.ACT_NAMES[w.act]
+    ws = torch.empty(moe.workspace_size(w.T, w.D, w.F, w.E, w.K, moe.F32, a), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty_like(x)
+    sel = torch.empty(w.T, w.K, dtype=torch.int64, device="cuda")
+    wt = torch.empty(w.T, w.K, dtype=torch.float32, device="cuda")
+
+    def fwd():
+        moe.ffn_forward(x, dev["router"], dev["gate_up_proj"], dev["down_proj"], w.E, w.K, True, a,
+                        out, sel, wt, dev["router_bias"], dev["b1"], dev["b2"], None, ws)
+
+    fwd()
+    torch.cuda.synchronize()
+    ref = (out.clone(), sel.clone(), wt.clone())
+    g = torch.cuda.CUDAGraph()
+    n0 = moe.kernel_launches()
+    with torch.cuda.graph(g):
+        fwd()
+    assert moe.kernel_launches() - n0 == 1
+    for _ in range(3):
+        out.zero_()
+        sel.zero_()
+        wt.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref[0]) and torch.equal(sel, ref[1]) and torch.equal(wt, ref[2])
+    assert moe.device_status() == moe.MOE_OK
+
+
 def test_kernel_launch_count_per_forward():
     """A forward launches router, scatter, gather, gate_up, down and combine;
     the scan kernel only runs for block-count tables of more than 4096
