@@ -589,6 +589,8 @@ SMALL_SPLIT_CASES = [
     (66, 40, 33, 47, 5, 2, "silu_gated", False),     # D, F not multiples of 4: 4-byte copies
     (67, 50, 8, 4, 2, 1, "silu_gated", True),        # F = 4: one column group, no split
     (68, 20, 12, 10, 1, 1, "relu", False),           # E = 1
+    (69, 10, 3, 5, 3, 2, "relu", False),             # D = 3: one lane holds all of D
+    (70, 16, 8, 1, 4, 2, "silu_gated", True),        # F = 1: a single column, never split
 ]
 
 
