@@ -15,8 +15,9 @@
 //      writes the routing outputs;
 //   2. from the rows each expert received, every CTA derives the same
 //      assignment of the C CTAs to experts: each expert with rows gets one
-//      CTA, and each further CTA goes to the expert with the most rows per
-//      CTA (lower index on ties).  An expert's s CTAs split its hidden
+//      CTA plus its proportional share of the rest (rounded down), and each
+//      CTA still free goes to the expert with the most rows per CTA (lower
+//      index on ties).  An expert's s CTAs split its hidden
 //      columns F into s slices of whole 4-column groups, so the routing skew
 //      of a real batch (one expert can take almost half of all rows) is
 //      spread over several SMs instead of setting the time of the launch;
@@ -50,9 +51,9 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRowGroup = 4;      // rows of one expert computed together by a thread
-constexpr int kLogitT = 2;        // router: tokens ...
-constexpr int kLogitE = 4;        // ... x experts computed together by a thread
-constexpr int kSplit = 8;         // router: lanes that split D for one (tokens, experts) block
+constexpr int kLogitT = 2;        // router: a block of kLogitT tokens ...
+constexpr int kLogitE = 4;        // ... x kLogitE experts ...
+constexpr int kSplit = 8;         // ... computed by kSplit lanes that split D between them
 
 struct SmallParams {
   const float* x;
