@@ -337,19 +337,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ void store_row32(__nv_bfloat16* rowp, int col0, int n_out,
-                                            const uint32_t (&w)[16]) {
-  uint4* dst = reinterpret_cast<uint4*>(rowp + col0);
-  if (col0 + 32 <= n_out) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-  } else {
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (col0 + 8 * q < n_out) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-  }
-}
-
 template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
