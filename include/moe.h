@@ -129,6 +129,12 @@ MOE_API size_t moe_ffn_workspace_size(int64_t T, int64_t D, int64_t F, int E, in
  * launched and no output is touched.  Returns MOE_OK once all kernels are
  * enqueued on `stream`; inputs must stay valid until the stream reaches
  * that point.
+ *
+ * A forward makes no synchronising call, so it can be recorded into a CUDA
+ * graph by stream capture.  The first call of a kernel variant on a device
+ * sets that kernel's attributes (and, for the one-kernel small layer,
+ * queries how large a cluster the device can co-schedule); make one call of
+ * the same shape outside capture first.
  */
 MOE_API moe_status_t moe_ffn_forward(const void* x, const void* router, const void* gate_up_proj,
                              const void* down_proj, int E, int K, int norm_topk_prob,
