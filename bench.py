@@ -626,6 +626,7 @@ def run_ours(args, w):
     build.build()
     moe.set_gemm_mode({"auto": moe.GEMM_AUTO, "1sm": moe.GEMM_1SM, "2sm": moe.GEMM_2SM}[args.gemm])
     moe.set_pdl(args.pdl)
+    moe.set_fused_gather(args.fused_gather)
     if args.tail_swap is not None:
         moe.set_tail_swap(args.tail_swap)
     tail_swap = moe.set_tail_swap(0)
@@ -754,6 +755,7 @@ def run_ours(args, w):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded, shapes of the published workloads; random-init weights)",
         "config": dict(workload_config(w, world), gemm=args.gemm, pdl=args.pdl, tail_swap=tail_swap,
+                       fused_gather=args.fused_gather,
                        **({"routing": {"score": args.score, "selection_bias_std": args.selection_bias,
                                        "dynamic_threshold": args.dynamic_threshold,
                                        "capacity_factor": args.capacity_factor,
@@ -895,6 +897,9 @@ def main(argv=None):
     ap.add_argument("--tail-swap", type=int, default=None,
                     help="rows up to which an expert's last CTA-pair tile runs with swapped "
                          "operands (0..255, 0 = off; default: the library's)")
+    ap.add_argument("--fused-gather", choices=["auto", "on", "off"], default="auto",
+                    help="bf16 gate_up fetches token rows from x by index (moe_set_fused_gather; "
+                         "default: the library's automatic choice)")
     ap.add_argument("--pdl", action="store_true",
                     help="launch the kernels with programmatic dependent launch (off by default)")
     ap.add_argument("--watchdog", type=float, default=120.0,

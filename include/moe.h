@@ -311,14 +311,24 @@ MOE_API int moe_set_small_cluster(int ctas);
 
 /*
  * Whether the bf16 gate_up GEMM fetches its token rows from x by index
- * (TMA tile::gather4, four rows per copy) instead of from an expert-sorted
- * copy written by a separate gather kernel.  Results are bit-identical.
- * Off by default: on B200 the four-row copies deliver the A operand far
- * slower than the tensor cores consume it (gate_up about 3x slower on the
- * Mixtral-shaped layer); it saves the gather kernel and its HBM write.
- * Returns the previous setting.
+ * (TMA tile::gather4, four rows per copy, only for the rows a tile holds)
+ * instead of from an expert-sorted copy written by a separate gather
+ * kernel.  Results are bit-identical either way.  Process-wide setting:
+ *   MOE_FUSED_GATHER_OFF  - always the expert-sorted copy;
+ *   MOE_FUSED_GATHER_ON   - always by index;
+ *   MOE_FUSED_GATHER_AUTO - (default) by index when the one-CTA GEMM runs
+ *                           and experts average at most 16 routed rows
+ *                           (decode steps): the few copies hide under the
+ *                           weight stream and the gather kernel is saved.
+ *                           With full tiles the four-row copies deliver A
+ *                           far slower than the tensor cores consume it
+ *                           (gate_up about 3x slower on the Mixtral layer).
+ * Returns the previous setting, or -1 for another value (nothing changes).
  */
-MOE_API int moe_set_fused_gather(int on);
+#define MOE_FUSED_GATHER_OFF 0
+#define MOE_FUSED_GATHER_ON 1
+#define MOE_FUSED_GATHER_AUTO 2
+MOE_API int moe_set_fused_gather(int mode);
 
 /*
  * Whether the kernels of one forward are launched with programmatic

@@ -223,22 +223,29 @@ __global__ void __launch_bounds__(THREADS, 1)
         rowB1 = rowB0 + 128;
       }
       int tok[4] = {0, 0, 0, 0};
+      // gathered A: only the lanes whose 4 rows hold some of this expert's
+      // rows fetch them; the other rows of the stage are padding (computed,
+      // never stored) and keep whatever the stage held
+      int gather_lanes = 32;
       if (GATHER) {
+        const int valid = min(BM, st->off[e + 1] - rowA);
+        gather_lanes = (valid + 3) >> 2;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int r = rowA + 4 * lane + i;
           tok[i] = r < rows_live ? __ldg(p.perm + r) / p.K : 0;   // rows past the end: any row
         }
       }
+      const uint32_t stage_tx = STAGE_BYTES - static_cast<uint32_t>(32 - gather_lanes) * 512u;
       bool ok = true;
       for (int kb = 0; kb < p.num_kb; ++kb) {
         int good = 1;
         if (lane == 0) {
           good = mbar_wait(&st->empty[stage], phase ^ 1u, abort, p.err, SITE_GEMM_PRODUCER) ? 1 : 0;
-          if (good) mbar_arrive_expect_tx(&st->full[stage], STAGE_BYTES);
+          if (good) mbar_arrive_expect_tx(&st->full[stage], stage_tx);
         }
         if (!__shfl_sync(0xffffffffu, good, 0)) { ok = false; break; }
-        if (GATHER)
+        if (GATHER && lane < gather_lanes)
           tma_gather4(&tmA, &st->full[stage], sA + stage * A_BYTES + lane * 512, kb * BK, tok[0],
                       tok[1], tok[2], tok[3]);
         if (lane == 0) {

@@ -29,7 +29,7 @@ thread_local std::string g_last_error;
 std::atomic<int> g_gemm_mode{MOE_GEMM_AUTO};
 std::atomic<int> g_tail_swap{MOE_TAIL_SWAP_DEFAULT};
 std::atomic<int> g_small_cluster{MOE_SMALL_CLUSTER_AUTO};
-std::atomic<int> g_fused_gather{0};
+std::atomic<int> g_fused_gather{MOE_FUSED_GATHER_AUTO};
 std::atomic<int> g_pdl{0};   // programmatic dependent launch: opt-in
 std::atomic<int> g_debug_sync_ms{0};   // > 0: bounded wait after every kernel of a forward
 // Block-count tables up to this many entries (blocks x experts) are scanned
@@ -344,7 +344,11 @@ extern "C" {
 
 int moe_abi_version(void) { return MOE_ABI_VERSION; }
 
-int moe_set_fused_gather(int on) { return g_fused_gather.exchange(on ? 1 : 0); }
+int moe_set_fused_gather(int mode) {
+  if (mode != MOE_FUSED_GATHER_OFF && mode != MOE_FUSED_GATHER_ON && mode != MOE_FUSED_GATHER_AUTO)
+    return -1;
+  return g_fused_gather.exchange(mode);
+}
 
 int moe_set_pdl(int on) { return g_pdl.exchange(on ? 1 : 0); }
 
@@ -526,8 +530,14 @@ moe_status_t ffn_forward_impl(const void* x, const void* router, const void* gat
   float* balance_out = opts ? opts->balance : nullptr;
   uint8_t* slot_kept = opts ? opts->slot_kept : nullptr;
   // bf16: gate_up reads the token rows of x directly (TMA gather), so the
-  // expert-sorted copy is not materialised
-  const bool fused_gather = dt == MOE_BF16 && g_fused_gather.load() != 0;
+  // expert-sorted copy is not materialised; automatically for layers on the
+  // one-CTA GEMM whose experts average at most 16 routed rows
+  const int fg_mode = g_fused_gather.load();
+  const bool pair_gemm = g_gemm_mode.load() == MOE_GEMM_2SM ||
+                         (g_gemm_mode.load() == MOE_GEMM_AUTO && T * K >= 512LL * E);
+  const bool fused_gather =
+      dt == MOE_BF16 && (fg_mode == MOE_FUSED_GATHER_ON ||
+                         (fg_mode == MOE_FUSED_GATHER_AUTO && !pair_gemm && T * K <= 16LL * E));
   const int Ti = static_cast<int>(T), Di = static_cast<int>(D), Fi = static_cast<int>(F);
   const int gu_act = act == MOE_ACT_SILU_GATED ? 0 : 1;
   const int gu_rows = act == MOE_ACT_SILU_GATED ? 2 * Fi : Fi;

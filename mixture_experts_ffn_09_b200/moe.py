@@ -417,10 +417,22 @@ def set_pdl(on: bool) -> bool:
     return bool(lib().moe_set_pdl(int(bool(on))))
 
 
-def set_fused_gather(on: bool) -> bool:
+FUSED_GATHER_OFF, FUSED_GATHER_ON, FUSED_GATHER_AUTO = 0, 1, 2
+
+
+def set_fused_gather(mode) -> int:
     """Selects whether the bf16 gate_up GEMM gathers its rows from x itself
-    (TMA gather4) or reads an expert-sorted copy; returns the previous."""
-    return bool(lib().moe_set_fused_gather(int(bool(on))))
+    (TMA gather4) or reads an expert-sorted copy: False/"off", True/"on" or
+    "auto" (the default; see moe_set_fused_gather in include/moe.h), or the
+    FUSED_GATHER_* value.  Returns the previous value (an int)."""
+    if isinstance(mode, str):
+        mode = {"off": FUSED_GATHER_OFF, "on": FUSED_GATHER_ON, "auto": FUSED_GATHER_AUTO}[mode]
+    elif isinstance(mode, bool):
+        mode = FUSED_GATHER_ON if mode else FUSED_GATHER_OFF
+    prev = int(lib().moe_set_fused_gather(int(mode)))
+    if prev < 0:
+        raise ValueError(f"fused gather mode must be 0, 1 or 2, not {mode}")
+    return prev
 
 
 def device_status(stream=None) -> int:

@@ -73,6 +73,18 @@ def test_process_wide_settings_validate_on_host(L):
         assert L.moe_set_gemm_mode(1) == 2
     finally:
         L.moe_set_gemm_mode(g)
+    f = L.moe_set_fused_gather(0)
+    try:
+        assert f == 2                              # MOE_FUSED_GATHER_AUTO
+        for bad in (3, -1, 7):
+            assert L.moe_set_fused_gather(bad) == -1
+        assert L.moe_set_fused_gather(1) == 0
+        assert moe.set_fused_gather("auto") == 1
+        assert moe.set_fused_gather(False) == 2 and moe.set_fused_gather(True) == 0
+        with pytest.raises(ValueError):
+            moe.set_fused_gather(5)
+    finally:
+        L.moe_set_fused_gather(f)
     c = L.moe_set_small_cluster(8)
     try:
         assert c == 0                              # MOE_SMALL_CLUSTER_AUTO

@@ -377,6 +377,38 @@ def test_fused_gather_equals_materialised_rows(gemm_mode, act):
         np.testing.assert_array_equal(a[k], b[k])
 
 
+@pytest.mark.parametrize("T,E,K,act", [(32, 8, 1, "silu_gated"), (40, 8, 2, "relu"),
+                                        (129, 1, 1, "silu_gated"), (300, 2, 1, "relu")])
+def test_fused_gather_on_partial_tiles(T, E, K, act):
+    """The one-CTA GEMM gathering token rows by index fetches only the rows a
+    tile holds (down to one); the rest of the stage is padding.  Off, on and
+    the automatic choice (on for these few-row layers, saving the gather
+    kernel) agree bit for bit, and all match the oracle."""
+    from mixture_experts_ffn_09_b200 import moe
+    d = synth.random_case(95 + T, T, 256, 384, E, act=act, dtype="bf16", weight_std=0.05)
+    dev = PL.to_device(d)
+    prev_mode = moe.set_gemm_mode(moe.GEMM_1SM)
+    prev = moe.set_fused_gather("off")
+    try:
+        g, _ = _full_check(d, E, K, True, act, "bf16")
+        res = {}
+        for mode in ("off", "on", "auto"):
+            moe.set_fused_gather(mode)
+            n0 = moe.kernel_launches()
+            res[mode] = PL.run_gpu(dev, E, K, True, act)
+            res[mode]["launches"] = moe.kernel_launches() - n0
+    finally:
+        moe.set_fused_gather(prev)
+        moe.set_gemm_mode(prev_mode)
+    for mode in ("on", "auto"):
+        for k in ("out", "sel", "w"):
+            np.testing.assert_array_equal(res[mode][k], res["off"][k])
+    np.testing.assert_array_equal(res["off"]["out"], g["out"])
+    assert res["on"]["launches"] == res["off"]["launches"] - 1          # no gather kernel
+    auto_on = T * K <= 16 * E
+    assert res["auto"]["launches"] == res["off"]["launches"] - (1 if auto_on else 0)
+
+
 @pytest.mark.parametrize("gemm_mode", MODES, indirect=True)
 def test_programmatic_dependent_launch_changes_nothing(gemm_mode):
     """The kernels give bit-identical results with and without programmatic
