@@ -60,11 +60,15 @@ def load_peaks() -> dict:
         return dict(FALLBACK_PEAKS)
 
 
-def source_hash() -> str:
-    """Hash of the grouped-GEMM source: a stored DRAM-traffic figure is only
+KERNEL_SOURCES = {"gate_up": ("gemm_tc.cu", "common.cuh"),          # one CTA per tile
+                  "gate_up_pair": ("gemm_tc2.cu", "common.cuh")}    # CTA pairs
+
+
+def source_hash(kernel: str) -> str:
+    """Hash of a grouped GEMM's sources: a stored DRAM-traffic figure is only
     reported while it matches the kernel it was taken on."""
     h = hashlib.sha256()
-    for f in ("gemm_tc.cu", "gemm_tc2.cu", "common.cuh"):
+    for f in KERNEL_SOURCES[kernel]:
         h.update(open(os.path.join(ROOT, "mixture_experts_ffn_09_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -74,7 +78,7 @@ def stored_traffic(workload: str, kernel: str):
     try:
         d = json.load(open(p))
         e = d[workload][kernel]
-        if e.get("source_hash") == source_hash():
+        if e.get("source_hash") == source_hash(kernel):
             return float(e["bytes_per_launch"])
     except Exception:
         pass
