@@ -648,6 +648,42 @@ def test_small_layer_split_over_the_cluster(seed, T, D, F, E, K, act, skew, clus
         assert (g["sel"][:, 0] == seed % E).all()
 
 
+def _random_small_layers(n, seed):
+    """Seeded small fp32 layers inside the one-kernel limits (E <= 8,
+    T*K <= 256, widths up to 48 so that the shared memory of any such layer
+    stays within the kernel's 200 KB), multiples of 4 or not."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        E = int(rng.integers(1, 9))
+        K = int(rng.integers(1, E + 1))
+        T = int(rng.integers(1, 256 // K + 1))
+        D = int(rng.integers(1, 49))
+        F = int(rng.integers(1, 49))
+        act = "relu" if rng.random() < 0.4 else "silu_gated"
+        skew = bool(rng.random() < 0.3)
+        out.append((T, D, F, E, K, act, skew))
+    return out
+
+
+@pytest.mark.parametrize("cluster", [8, 16])
+@pytest.mark.parametrize("T,D,F,E,K,act,skew", _random_small_layers(10, 4242))
+def test_small_layer_random_sweep(T, D, F, E, K, act, skew, cluster):
+    """Seeded random small fp32 layers through the one-kernel path, with
+    clusters of 8 and 16 CTAs: every token against the oracle, one launch."""
+    from mixture_experts_ffn_09_b200 import moe
+    seed = 7000 + T + D + F + E
+    d = _skewed_small(seed, T, D, F, E, act, seed % E) if skew else \
+        synth.random_case(seed, T, D, F, E, act=act, dtype="f32", weight_std=0.3)
+    prev = moe.set_small_cluster(cluster)
+    try:
+        n0 = moe.kernel_launches()
+        _full_check(d, E, K, True, act, "f32")
+        assert moe.kernel_launches() - n0 == 1
+    finally:
+        moe.set_small_cluster(prev)
+
+
 @pytest.mark.parametrize("act", ["silu_gated", "relu"])
 def test_split_last_wave(act):
     """Layers in the CTA-pair regime run their last wave as k-halves: the
